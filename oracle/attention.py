@@ -1,0 +1,151 @@
+"""Float64 CPU oracle of the fused attention forward  out = softmax(z + B) V.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  It shares no code
+with the CUDA library and the library never calls it.
+
+It is the plain definition, written out in float64 per (batch, query head),
+in blocks of query rows so that memory stays bounded:
+
+* Score (page "어텐션 메커니즘" §2; page "SDPA란 무엇인가" §1, the
+  softmax(QK^T/sqrt(E) + B)V formula and its four steps):
+    dot  z_ij = scale * <q_i, k_j>
+    rbf  z_ij = -scale * ||q_i - k_j||^2 + scale * ||q_i||^2
+  The RBF distance is computed directly, element by element (page
+  "Dot-Product Attention을 거리 기반 RBF-Attention으로 교체한 실험기",
+  섹션별 상세: distance attention, torch.cdist form).  The + scale*||q_i||^2
+  term fixes the logit frame to the expanded form 2*scale*<q,k> -
+  scale*||k||^2 that the same page derives by shift invariance; it cancels in
+  any softmax without a sink and only matters when a sink logit competes.
+* Mask (page "SDPA란 무엇인가" §1 bias B in {0, -inf}; §4 trap 3 causal
+  alignment; page "어텐션 메커니즘" §5 causal mask, §6 sliding window):
+  with the bottom-right alignment i' = i + (S - L),
+    causal  key j visible iff j <= i'
+    window  key j visible iff 0 <= i' - j < W   (W keys, self included)
+  and an additive bias B[i, j] (0 or -inf) composes with either.
+* Grouped-query attention (page "SDPA란 무엇인가" §5): query head hq reads
+  KV head hq // (Hq // H).
+* Sink (page "Attention Sink" §4.2, §5.2-5.4): a per-query-head logit s_h
+  enters the softmax denominator and not the value sum.  With A the visible
+  keys:  M = max(max_{j in A} z_j, s),  D = e^{s-M} + sum_{j in A} e^{z_j-M},
+  out = sum_{j in A} e^{z_j-M} v_j / D,  lse = M + ln D.
+* A row with no visible key and no sink gives out = 0 and lse = -inf (page
+  "SDPA란 무엇인가" §4: SDPA returns 0 instead of NaN for a fully masked row).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+
+def visible(rows: np.ndarray, S: int, L: int, mask_kind: str, window: int = 0) -> np.ndarray:
+    """Boolean (R, S) visibility of keys 0..S-1 for query positions ``rows``.
+
+    Bottom-right alignment: query i sits at key position i' = i + (S - L).
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    ip = rows[:, None] + (S - L)
+    j = np.arange(S, dtype=np.int64)[None, :]
+    if mask_kind == "none":
+        return np.ones((rows.size, S), dtype=bool)
+    if mask_kind == "causal":
+        return j <= ip
+    if mask_kind == "window":
+        if window < 1:
+            raise ValueError("window must be >= 1")
+        d = ip - j
+        return (d >= 0) & (d < window)
+    raise ValueError(f"unknown mask kind {mask_kind!r}")
+
+
+def logits(q_rows: np.ndarray, k: np.ndarray, scale: float, mode: str, key_block: int = 512) -> np.ndarray:
+    """Unmasked logits z (R, S) in float64."""
+    q_rows = np.asarray(q_rows, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    if mode == "dot":
+        return scale * (q_rows @ k.T)
+    if mode == "rbf":
+        R, S = q_rows.shape[0], k.shape[0]
+        d2 = np.empty((R, S), dtype=np.float64)
+        # direct squared distance, sum over e of (q_e - k_e)^2
+        for j0 in range(0, S, key_block):
+            diff = q_rows[:, None, :] - k[None, j0:j0 + key_block, :]
+            d2[:, j0:j0 + key_block] = np.einsum("rse,rse->rs", diff, diff)
+        qn = np.einsum("re,re->r", q_rows, q_rows)
+        return -scale * d2 + scale * qn[:, None]
+    raise ValueError(f"unknown mode {mode!r}")
+
+
+def softmax_with_sink(z: np.ndarray, vis: np.ndarray, sink: float | None):
+    """Weights alpha (R, S), sink probability (R,), lse (R,) from masked logits.
+
+    ``z`` already carries the additive bias; ``vis`` marks keys the mask kind
+    leaves visible.  Keys with z = -inf (from the bias) get weight 0.
+    """
+    zm = np.where(vis, z, NEG_INF)
+    s = NEG_INF if sink is None else float(sink)
+    M = np.maximum(np.max(zm, axis=1, initial=NEG_INF), s)
+    finite = np.isfinite(M)
+    Ms = np.where(finite, M, 0.0)
+    e = np.where(np.isfinite(zm), np.exp(zm - Ms[:, None]), 0.0)
+    es = np.exp(s - Ms) if np.isfinite(s) else np.zeros_like(Ms)
+    D = es + e.sum(axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        alpha = np.where(finite[:, None], e / np.where(finite, D, 1.0)[:, None], 0.0)
+        p_sink = np.where(finite, es / np.where(finite, D, 1.0), 0.0)
+        lse = np.where(finite, Ms + np.log(np.where(finite, D, 1.0)), NEG_INF)
+    return alpha, p_sink, lse
+
+
+def attend_rows(q_rows, rows, k, v, L, *, scale, mode="dot", sink=None, mask_kind="none",
+                window=0, bias_rows=None, return_weights=False):
+    """Attention of query rows ``q_rows`` (R, E) at positions ``rows`` against one KV head.
+
+    k (S, E), v (S, Ev), bias_rows (R, S) or None.  Returns out (R, Ev) and
+    lse (R,) (and the weights and sink probability when asked).
+    """
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    S = k.shape[0]
+    z = logits(q_rows, k, scale, mode)
+    if bias_rows is not None:
+        z = z + np.asarray(bias_rows, dtype=np.float64)
+    vis = visible(rows, S, L, mask_kind, window)
+    alpha, p_sink, lse = softmax_with_sink(z, vis, sink)
+    out = alpha @ v
+    if return_weights:
+        return out, lse, alpha, p_sink
+    return out, lse
+
+
+def attention_forward(q, k, v, *, scale, mode="dot", sink=None, mask_kind="none", window=0,
+                      bias=None, row_block=128):
+    """Whole forward: q (N,Hq,L,E), k (N,H,S,E), v (N,H,S,Ev) float64.
+
+    sink: per-query-head logits (Hq,) or None.  bias: (L, S) or None.
+    Returns out (N,Hq,L,Ev) and lse (N,Hq,L).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    N, Hq, L, _ = q.shape
+    H = k.shape[1]
+    if Hq % H:
+        raise ValueError("Hq must be a multiple of H")
+    g = Hq // H
+    Ev = v.shape[3]
+    out = np.zeros((N, Hq, L, Ev), dtype=np.float64)
+    lse = np.zeros((N, Hq, L), dtype=np.float64)
+    for n in range(N):
+        for hq in range(Hq):
+            kvh = hq // g
+            s = None if sink is None else float(sink[hq])
+            for i0 in range(0, L, row_block):
+                rows = np.arange(i0, min(L, i0 + row_block))
+                b = None if bias is None else np.asarray(bias)[rows]
+                o, l = attend_rows(q[n, hq, rows], rows, k[n, kvh], v[n, kvh], L, scale=scale,
+                                   mode=mode, sink=s, mask_kind=mask_kind, window=window,
+                                   bias_rows=b)
+                out[n, hq, rows] = o
+                lse[n, hq, rows] = l
+    return out, lse

@@ -1,0 +1,355 @@
+"""Pins of the float64 oracle: each check compares the oracle with something
+other than itself (a value a page prints, a closed form, an invariant, a
+library routine the definition reduces to, or pure-Python brute force).
+
+Each ``check_*`` raises AssertionError on a mismatch.  ``test_oracle_pins.py``
+runs them against the oracle; ``test_oracle_mutations.py`` plants plausible
+mistakes in the oracle and shows that some check catches each one.
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+from torch.nn.attention.bias import causal_lower_right
+
+from oracle import attention as orc
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+# ----------------------------------------------------------------------------
+# the dot-product path reduces to a library routine: torch SDPA in float64
+# ----------------------------------------------------------------------------
+
+def check_dot_matches_sdpa(seed=0):
+    rng = np.random.default_rng(seed)
+    cases = [
+        # N, Hq, H, L, S, E, Ev, mask
+        (2, 4, 4, 9, 9, 8, 6, "none"),
+        (1, 4, 2, 7, 13, 8, 8, "causal"),      # L != S: bottom-right alignment
+        (2, 6, 2, 11, 11, 16, 4, "causal"),    # GQA g = 3
+        (1, 2, 1, 5, 12, 4, 4, "bias"),
+    ]
+    for N, Hq, H, L, S, E, Ev, mask in cases:
+        q, k, v = _rand(rng, N, Hq, L, E), _rand(rng, N, H, S, E), _rand(rng, N, H, S, Ev)
+        scale = 0.37
+        bias = None
+        kw = {}
+        if mask == "causal":
+            kw["attn_mask"] = causal_lower_right(L, S)
+        elif mask == "bias":
+            b = np.where(rng.random((L, S)) < 0.3, -np.inf, 0.0)
+            b[:, -1] = 0.0  # keep each row non-empty
+            bias = b
+            kw["attn_mask"] = torch.from_numpy(b)
+        ref = F.scaled_dot_product_attention(
+            torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v),
+            scale=scale, enable_gqa=(Hq != H), **kw).numpy()
+        out, _ = orc.attention_forward(q, k, v, scale=scale, mode="dot",
+                                       mask_kind="causal" if mask == "causal" else "none",
+                                       bias=bias)
+        err = np.max(np.abs(out - ref))
+        assert err < 1e-12, (mask, err)
+
+
+# ----------------------------------------------------------------------------
+# brute force with pure-Python loops on tiny inputs (every mode, mask, sink)
+# ----------------------------------------------------------------------------
+
+def _brute_row(qi, i, K, V, L, scale, mode, sink, mask_kind, window, brow):
+    S = len(K)
+    ip = i + (S - L)
+    zs, vs = [], []
+    for j in range(S):
+        if mask_kind == "causal" and j > ip:
+            continue
+        if mask_kind == "window" and not (0 <= ip - j < window):
+            continue
+        if mode == "dot":
+            z = scale * math.fsum(a * b for a, b in zip(qi, K[j]))
+        else:
+            z = -scale * math.fsum((a - b) ** 2 for a, b in zip(qi, K[j])) \
+                + scale * math.fsum(a * a for a in qi)
+        if brow is not None:
+            z += brow[j]
+        if z == -math.inf:
+            continue
+        zs.append(z)
+        vs.append(V[j])
+    cands = zs + ([sink] if sink is not None else [])
+    if not cands:
+        return [0.0] * len(V[0]), -math.inf
+    M = max(cands)
+    ws = [math.exp(z - M) for z in zs]
+    D = math.fsum(ws) + (math.exp(sink - M) if sink is not None else 0.0)
+    out = [math.fsum(w * vj[d] for w, vj in zip(ws, vs)) / D for d in range(len(V[0]))]
+    return out, M + math.log(D)
+
+
+def check_brute_force(seed=1):
+    rng = np.random.default_rng(seed)
+    for mode in ("dot", "rbf"):
+        for mask_kind, window in (("none", 0), ("causal", 0), ("window", 2), ("window", 1)):
+            for sink in (None, 0.3, -2.0):
+                for L, S in ((4, 4), (2, 5), (5, 3)):
+                    E, Ev = 3, 2
+                    q, k, v = _rand(rng, 1, 2, L, E), _rand(rng, 1, 1, S, E), _rand(rng, 1, 1, S, Ev)
+                    bias = np.where(rng.random((L, S)) < 0.2, -np.inf, 0.0)
+                    sk = None if sink is None else np.array([sink, sink + 0.5])
+                    out, lse = orc.attention_forward(q, k, v, scale=0.6, mode=mode, sink=sk,
+                                                     mask_kind=mask_kind, window=window, bias=bias)
+                    for hq in range(2):
+                        s = None if sk is None else float(sk[hq])
+                        for i in range(L):
+                            bo, bl = _brute_row(list(q[0, hq, i]), i, k[0, 0].tolist(), v[0, 0].tolist(),
+                                                L, 0.6, mode, s, mask_kind, window, bias[i].tolist())
+                            assert np.allclose(out[0, hq, i], bo, rtol=0, atol=1e-12), (mode, mask_kind, sink)
+                            if bl == -math.inf:
+                                assert lse[0, hq, i] == -np.inf
+                            else:
+                                assert abs(lse[0, hq, i] - bl) < 1e-12, (mode, mask_kind, sink)
+
+
+# ----------------------------------------------------------------------------
+# RBF: the expansion identity, and the two temperature limits
+# ----------------------------------------------------------------------------
+
+def check_rbf_expansion(seed=2):
+    """Direct -scale*||q-k||^2 (+ scale*||q||^2 frame) equals the expanded
+    2*scale*q.k - scale*||k||^2 (the expansion -||q||^2 - ||k||^2 + 2 q.k with
+    the query norm dropped by shift invariance)."""
+    rng = np.random.default_rng(seed)
+    q, k = _rand(rng, 7, 16) * 3, _rand(rng, 11, 16) * 2
+    scale = 0.125
+    z = orc.logits(q, k, scale, "rbf")
+    expanded = scale * (2.0 * np.einsum("re,se->rs", q, k) - np.einsum("se,se->s", k, k)[None, :])
+    rel = np.max(np.abs(z - expanded)) / np.max(np.abs(expanded))
+    assert rel < 1e-12, rel
+
+
+def check_rbf_limits(seed=3):
+    rng = np.random.default_rng(seed)
+    L, S, E, Ev = 6, 9, 5, 4
+    q, k, v = _rand(rng, 1, 1, L, E), _rand(rng, 1, 1, S, E), _rand(rng, 1, 1, S, Ev)
+    for mask_kind in ("none", "causal"):
+        vis = orc.visible(np.arange(L), S, L, mask_kind)
+        # scale -> 0: uniform over visible keys -> mean of visible value rows
+        out, _ = orc.attention_forward(q, k, v, scale=1e-13, mode="rbf", mask_kind=mask_kind)
+        for i in range(L):
+            mean = v[0, 0][vis[i]].mean(axis=0)
+            assert np.allclose(out[0, 0, i], mean, atol=1e-9)
+        # scale -> inf: one-hot on the nearest visible key (brute-force argmin)
+        out, _ = orc.attention_forward(q, k, v, scale=1e4, mode="rbf", mask_kind=mask_kind)
+        for i in range(L):
+            best, bj = math.inf, -1
+            for j in range(S):
+                if not vis[i, j]:
+                    continue
+                d = sum((a - b) ** 2 for a, b in zip(q[0, 0, i], k[0, 0, j]))
+                if d < best:
+                    best, bj = d, j
+            assert np.allclose(out[0, 0, i], v[0, 0, bj], atol=1e-9)
+
+
+def check_dot_limits(seed=4):
+    """scale -> 0: weights uniform over visible keys, lse = ln(n_vis) (ln(n_vis + e^s) with a sink)."""
+    rng = np.random.default_rng(seed)
+    L, S, E, Ev = 5, 8, 4, 3
+    q, k, v = _rand(rng, 1, 1, L, E), _rand(rng, 1, 1, S, E), _rand(rng, 1, 1, S, Ev)
+    for sink in (None, 0.7):
+        sk = None if sink is None else np.array([sink])
+        out, lse = orc.attention_forward(q, k, v, scale=1e-15, mode="dot", mask_kind="causal", sink=sk)
+        for i in range(L):
+            nvis = i + (S - L) + 1
+            extra = 0.0 if sink is None else math.exp(sink)
+            assert abs(lse[0, 0, i] - math.log(nvis + extra)) < 1e-12
+            mean = v[0, 0, :nvis].mean(axis=0) * nvis / (nvis + extra)
+            assert np.allclose(out[0, 0, i], mean, atol=1e-12)
+
+
+def check_uniform_entropy_golden():
+    """Golden: n = 24 tokens, temperature -> inf: mean row entropy ln 24 = 3.178."""
+    g = _golden("uniform_entropy_n24.json")
+    n = g["n"]
+    rng = np.random.default_rng(5)
+    x = _rand(rng, n, 2)
+    rows = np.arange(n)
+    _, _, alpha, _ = orc.attend_rows(x, rows, x, x, n, scale=1e-12, mode="dot", return_weights=True)
+    ent = float(np.mean(-np.sum(alpha * np.log(alpha), axis=1)))
+    assert round(ent, g["decimals"]) == g["entropy"], ent
+
+
+# ----------------------------------------------------------------------------
+# sink
+# ----------------------------------------------------------------------------
+
+def check_sink_limit(seed=6):
+    rng = np.random.default_rng(seed)
+    q, k, v = _rand(rng, 1, 2, 6, 4), _rand(rng, 1, 1, 6, 4), _rand(rng, 1, 1, 6, 3)
+    for mode in ("dot", "rbf"):
+        ref, rl = orc.attention_forward(q, k, v, scale=0.5, mode=mode, mask_kind="causal")
+        for s in (-np.inf, -1e30):
+            out, lse = orc.attention_forward(q, k, v, scale=0.5, mode=mode, mask_kind="causal",
+                                             sink=np.array([s, s]))
+            assert np.array_equal(out, ref) and np.array_equal(lse, rl), (mode, s)
+
+
+def check_sink_mass(seed=7):
+    """Weights sum to 1 - p_sink, p_sink = e^{s - lse}; out = (1 - p_sink) * out_without_sink."""
+    rng = np.random.default_rng(seed)
+    L, S = 5, 7
+    q, k, v = _rand(rng, L, 4), _rand(rng, S, 4), _rand(rng, S, 3)
+    rows = np.arange(L)
+    for mode in ("dot", "rbf"):
+        for s in (-1.0, 0.0, 2.5):
+            out, lse, alpha, ps = orc.attend_rows(q, rows, k, v, L, scale=0.4, mode=mode, sink=s,
+                                                  mask_kind="causal", return_weights=True)
+            base, _ = orc.attend_rows(q, rows, k, v, L, scale=0.4, mode=mode, mask_kind="causal")
+            assert np.all(alpha >= 0)
+            assert np.allclose(alpha.sum(axis=1), 1.0 - ps, atol=1e-14)
+            assert np.allclose(ps, np.exp(s - lse), atol=1e-14)
+            assert np.allclose(out, (1.0 - ps)[:, None] * base, atol=1e-13)
+
+
+def check_zero_sink_equivalence(seed=8):
+    """R zero K/V rows prepended (and visible to every query) equal no registers
+    plus a sink logit ln R: a zero key has logit exactly 0 in both score modes,
+    i.e. adding e^0 = 1 to the denominator per register (page 'Attention Sink'
+    §3.3 zero sink; register tokens of the RBF page)."""
+    rng = np.random.default_rng(seed)
+    L, E, Ev = 6, 5, 4
+    for R in (1, 4):
+        for mode in ("dot", "rbf"):
+            for mask_kind in ("none", "causal"):
+                q = _rand(rng, 1, 2, L, E)
+                k, v = _rand(rng, 1, 1, L, E), _rand(rng, 1, 1, L, Ev)
+                kr = np.concatenate([np.zeros((1, 1, R, E)), k], axis=2)
+                vr = np.concatenate([np.zeros((1, 1, R, Ev)), v], axis=2)
+                with_regs, _ = orc.attention_forward(q, kr, vr, scale=0.3, mode=mode, mask_kind=mask_kind)
+                sinked, _ = orc.attention_forward(q, k, v, scale=0.3, mode=mode, mask_kind=mask_kind,
+                                                  sink=np.full(2, math.log(R)))
+                assert np.allclose(with_regs, sinked, atol=1e-13), (R, mode, mask_kind)
+
+
+# ----------------------------------------------------------------------------
+# convexity, masks, structure
+# ----------------------------------------------------------------------------
+
+def check_convexity(seed=9):
+    rng = np.random.default_rng(seed)
+    L, S = 8, 8
+    q, k, v = _rand(rng, L, 6) * 2, _rand(rng, S, 6), _rand(rng, S, 5)
+    rows = np.arange(L)
+    for mode in ("dot", "rbf"):
+        for mask_kind, w in (("none", 0), ("causal", 0), ("window", 3)):
+            out, _, alpha, _ = orc.attend_rows(q, rows, k, v, L, scale=0.9, mode=mode,
+                                               mask_kind=mask_kind, window=w, return_weights=True)
+            vis = orc.visible(rows, S, L, mask_kind, w)
+            assert np.all(alpha >= 0) and np.all(alpha[~vis] == 0)
+            assert np.allclose(alpha.sum(axis=1), 1.0, atol=1e-14)
+            for i in range(L):
+                vv = v[vis[i]]
+                assert np.all(out[i] >= vv.min(axis=0) - 1e-14)
+                assert np.all(out[i] <= vv.max(axis=0) + 1e-14)
+
+
+def check_causal_alignment_golden():
+    g = _golden("causal_alignment_L1_S6.json")
+    L, S = g["L"], g["S"]
+    br = orc.visible(np.array([0]), S, L, "causal")[0]
+    assert br.tolist() == g["bottom_right_row"]
+    # the top-left alignment is the same rule with the offset S - L taken as 0
+    tl = orc.visible(np.array([0]), S, S, "causal")[0]
+    assert tl.tolist() == g["top_left_row"]
+    assert causal_lower_right(L, S)._materialize().tolist()[0] == g["bottom_right_row"]
+
+
+def check_fully_masked_rows(seed=10):
+    """A row whose keys are all masked gives out = 0 (as SDPA returns), lse = -inf;
+    with a sink, out = 0 and lse = s."""
+    rng = np.random.default_rng(seed)
+    L, S = 4, 5
+    q, k, v = _rand(rng, 1, 1, L, 3), _rand(rng, 1, 1, S, 3), _rand(rng, 1, 1, S, 2)
+    bias = np.zeros((L, S))
+    bias[2, :] = -np.inf
+    out, lse = orc.attention_forward(q, k, v, scale=0.5, bias=bias)
+    ref = F.scaled_dot_product_attention(torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v),
+                                         attn_mask=torch.from_numpy(bias), scale=0.5).numpy()
+    assert np.all(out[0, 0, 2] == 0.0) and lse[0, 0, 2] == -np.inf
+    assert np.max(np.abs(out - ref)) < 1e-12
+    out, lse = orc.attention_forward(q, k, v, scale=0.5, bias=bias, sink=np.array([0.25]))
+    assert np.all(out[0, 0, 2] == 0.0) and lse[0, 0, 2] == 0.25
+    # L > S with causal: rows i < L - S see no key
+    q2 = _rand(rng, 1, 1, 6, 3)
+    out, lse = orc.attention_forward(q2, k[:, :, :3], v[:, :, :3], scale=0.5, mask_kind="causal")
+    assert np.all(out[0, 0, :3] == 0.0) and np.all(lse[0, 0, :3] == -np.inf)
+    assert np.all(np.isfinite(lse[0, 0, 3:]))
+
+
+def check_window_semantics(seed=11):
+    rng = np.random.default_rng(seed)
+    L, S = 7, 10
+    q, k, v = _rand(rng, 1, 1, L, 4), _rand(rng, 1, 1, S, 4), _rand(rng, 1, 1, S, 3)
+    # W = 1: each query sees only its own aligned key i' = i + S - L
+    out, _ = orc.attention_forward(q, k, v, scale=0.8, mask_kind="window", window=1)
+    for i in range(L):
+        assert np.array_equal(out[0, 0, i], v[0, 0, i + S - L])
+    # W >= S: identical to causal
+    a, la = orc.attention_forward(q, k, v, scale=0.8, mask_kind="window", window=S)
+    b, lb = orc.attention_forward(q, k, v, scale=0.8, mask_kind="causal")
+    assert np.array_equal(a, b) and np.array_equal(la, lb)
+    # exactly min(W, i'+1) keys visible
+    for W in (2, 3, 5):
+        vis = orc.visible(np.arange(L), S, L, "window", W)
+        for i in range(L):
+            assert vis[i].sum() == min(W, i + S - L + 1)
+
+
+def check_permutation_equivariance(seed=12):
+    rng = np.random.default_rng(seed)
+    L, S = 6, 9
+    q, k, v = _rand(rng, 1, 1, L, 4), _rand(rng, 1, 1, S, 4), _rand(rng, 1, 1, S, 3)
+    for mode in ("dot", "rbf"):
+        base, bl = orc.attention_forward(q, k, v, scale=0.7, mode=mode)
+        pk = rng.permutation(S)
+        o, l_ = orc.attention_forward(q, k[:, :, pk], v[:, :, pk], scale=0.7, mode=mode)
+        assert np.allclose(o, base, atol=1e-13) and np.allclose(l_, bl, atol=1e-13)
+        pq = rng.permutation(L)
+        o, l_ = orc.attention_forward(q[:, :, pq], k, v, scale=0.7, mode=mode)
+        assert np.allclose(o, base[:, :, pq], atol=1e-13) and np.allclose(l_, bl[:, :, pq], atol=1e-13)
+
+
+def check_gqa_repeat(seed=13):
+    rng = np.random.default_rng(seed)
+    N, Hq, H, L, S = 2, 6, 2, 5, 7
+    q, k, v = _rand(rng, N, Hq, L, 4), _rand(rng, N, H, S, 4), _rand(rng, N, H, S, 3)
+    sink = rng.standard_normal(Hq)
+    for mode in ("dot", "rbf"):
+        a, la = orc.attention_forward(q, k, v, scale=0.5, mode=mode, mask_kind="causal", sink=sink)
+        kr, vr = np.repeat(k, Hq // H, axis=1), np.repeat(v, Hq // H, axis=1)
+        b, lb = orc.attention_forward(q, kr, vr, scale=0.5, mode=mode, mask_kind="causal", sink=sink)
+        assert np.array_equal(a, b) and np.array_equal(la, lb)
+
+
+ALL_CHECKS = [
+    check_dot_matches_sdpa, check_brute_force, check_rbf_expansion, check_rbf_limits,
+    check_dot_limits, check_uniform_entropy_golden, check_sink_limit, check_sink_mass,
+    check_zero_sink_equivalence, check_convexity, check_causal_alignment_golden,
+    check_fully_masked_rows, check_window_semantics, check_permutation_equivariance,
+    check_gqa_repeat,
+]

@@ -1,0 +1,97 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and show a pin catches each."""
+
+import numpy as np
+import pytest
+
+import oracle_pins as pins
+from oracle import attention as orc
+
+_real_logits = orc.logits
+_real_visible = orc.visible
+_real_softmax = orc.softmax_with_sink
+
+
+def _rbf_direct_frame(q_rows, k, scale, mode, key_block=512):
+    z = _real_logits(q_rows, k, scale, mode, key_block)
+    if mode == "rbf":  # drop the +scale*||q||^2 frame term
+        z = z - scale * np.einsum("re,re->r", q_rows, q_rows)[:, None]
+    return z
+
+
+def _rbf_sign_flip(q_rows, k, scale, mode, key_block=512):
+    z = _real_logits(q_rows, k, scale, mode, key_block)
+    if mode == "rbf":
+        qn = scale * np.einsum("re,re->r", q_rows, q_rows)[:, None]
+        z = -(z - qn) + qn
+    return z
+
+
+def _dot_scale_dropped(q_rows, k, scale, mode, key_block=512):
+    if mode == "dot":
+        return q_rows @ k.T
+    return _real_logits(q_rows, k, scale, mode, key_block)
+
+
+def _top_left(rows, S, L, mask_kind, window=0):
+    return _real_visible(rows, S, S, mask_kind, window)
+
+
+def _window_off_by_one(rows, S, L, mask_kind, window=0):
+    if mask_kind == "window":
+        rows = np.asarray(rows)
+        d = rows[:, None] + (S - L) - np.arange(S)[None, :]
+        return (d >= 0) & (d <= window)
+    return _real_visible(rows, S, L, mask_kind, window)
+
+
+def _sink_in_values(z, vis, sink):
+    alpha, ps, lse = _real_softmax(z, vis, sink)
+    if sink is not None and alpha.shape[1]:
+        alpha = alpha.copy()
+        alpha[:, 0] += ps  # sink mass leaks into the first value row
+    return alpha, ps, lse
+
+
+def _lse_without_sink(z, vis, sink):
+    alpha, ps, lse = _real_softmax(z, vis, sink)
+    _, _, lse0 = _real_softmax(z, vis, None)
+    return alpha, ps, lse0 if sink is not None else lse
+
+
+MUTATIONS = [
+    ("logits", _rbf_direct_frame, pins.check_zero_sink_equivalence),
+    ("logits", _rbf_direct_frame, pins.check_rbf_expansion),
+    ("logits", _rbf_sign_flip, pins.check_rbf_limits),
+    ("logits", _dot_scale_dropped, pins.check_dot_matches_sdpa),
+    ("visible", _top_left, pins.check_causal_alignment_golden),
+    ("visible", _top_left, pins.check_dot_matches_sdpa),
+    ("visible", _window_off_by_one, pins.check_window_semantics),
+    ("softmax_with_sink", _sink_in_values, pins.check_sink_mass),
+    ("softmax_with_sink", _lse_without_sink, pins.check_brute_force),
+]
+
+
+@pytest.mark.parametrize("attr,bad,check", MUTATIONS,
+                         ids=[f"{a}:{b.__name__}->{c.__name__}" for a, b, c in MUTATIONS])
+def test_planted_mistake_is_caught(monkeypatch, attr, bad, check):
+    monkeypatch.setattr(orc, attr, bad)
+    with pytest.raises(AssertionError):
+        check()
+
+
+def test_gqa_head_map_mistake_is_caught(monkeypatch):
+    """Reading KV head hq % H instead of hq // (Hq/H) is caught by the SDPA pin."""
+    real_forward = orc.attention_forward
+
+    def forward_modulo(q, k, v, **kw):
+        q = np.asarray(q)
+        Hq, H = q.shape[1], k.shape[1]
+        perm = [hq % H for hq in range(Hq)]
+        # emulate the wrong map by handing each query head the KV head hq % H
+        kk = np.asarray(k)[:, perm]
+        vv = np.asarray(v)[:, perm]
+        return real_forward(q, kk, vv, **kw)
+
+    monkeypatch.setattr(orc, "attention_forward", forward_modulo)
+    with pytest.raises(AssertionError):
+        pins.check_dot_matches_sdpa()

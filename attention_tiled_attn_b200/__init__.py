@@ -1,0 +1,143 @@
+"""Fused attention forward for NVIDIA B200 (sm_100a): Python binding.
+
+A thin ctypes layer over the C ABI declared in ``include/attn_b200.h``.  It only
+marshals arguments (shapes, dtypes, data pointers, the current CUDA stream);
+every step of the computation runs in the library's CUDA kernels.  There is
+no CPU fallback: without the built library or a CUDA device the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libattn_b200.so")
+
+MODES = {"dot": 0, "rbf": 1, "sink": 2}
+MASKS = {"none": 0, "causal": 1, "window": 2}
+DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+
+ATTN_OK = 0
+
+
+class AttnError(RuntimeError):
+    """A non-zero status returned by the library."""
+
+    def __init__(self, status: int, text: str):
+        super().__init__(f"attn status {status}: {text}")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"CUDA library not built: {path} is missing (run python -m attention_tiled_attn_b200.build)")
+    lib = ctypes.CDLL(path)
+    vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp, ci, vp]
+    lib.attn_fwd.restype = ci
+    lib.attn_status_string.argtypes = [ci]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_release_workspace.argtypes = []
+    lib.attn_release_workspace.restype = None
+    lib.attn_device_status.argtypes = [vp]
+    lib.attn_device_status.restype = ci
+    lib.attn_version.argtypes = []
+    lib.attn_version.restype = ci
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().attn_status_string(int(status)).decode()
+
+
+def _check(status: int):
+    if status != ATTN_OK:
+        raise AttnError(status, status_string(status))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def attn_fwd_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H, L, S, E, Ev, scale, mode, sink_ptr,
+                 mask_kind, window, bias_ptr, dtype, stream_ptr) -> int:
+    """The C entry point with integer pointers; returns the status code."""
+    lib = load_library()
+    c = lambda p: None if p is None else ctypes.c_void_p(int(p))  # noqa: E731
+    return lib.attn_fwd(c(q_ptr), c(k_ptr), c(v_ptr), c(out_ptr), c(lse_ptr), int(N), int(Hq), int(H), int(L),
+                        int(S), int(E), int(Ev), float(scale), int(mode), c(sink_ptr), int(mask_kind),
+                        int(window), c(bias_ptr), int(dtype), c(stream_ptr))
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float, mode: str = "dot",
+             sink: torch.Tensor | None = None, mask_kind: str = "none", window: int = 0,
+             bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+             lse: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None):
+    """out = softmax(z + B) V on the GPU.  Returns (out, lse).
+
+    q (N, Hq, L, E), k (N, H, S, E), v (N, H, S, Ev): contiguous CUDA tensors,
+    all bfloat16 or all float32.  sink: (Hq,) float32 or None.  bias: (L, S)
+    float32 or None.  mode: "dot", "rbf" or "sink"; mask_kind: "none",
+    "causal" or "window".  out/lse may be given (contiguous, right shape).
+    """
+    load_library()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 4-D tensor")
+    if q.dtype not in DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share dtype bfloat16 or float32")
+    N, Hq, L, E = q.shape
+    Nk, H, S, Ek = k.shape
+    Nv, Hv, Sv, Ev = v.shape
+    if Nk != N or Nv != N or Hv != H or Sv != S or Ek != E:
+        raise ValueError("inconsistent q/k/v shapes")
+    if sink is not None and (sink.dtype != torch.float32 or sink.numel() != Hq or not sink.is_cuda
+                             or not sink.is_contiguous()):
+        raise ValueError("sink must be a contiguous CUDA float32 tensor of Hq values")
+    if bias is not None and (bias.dtype != torch.float32 or tuple(bias.shape) != (L, S) or not bias.is_cuda
+                             or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous CUDA float32 (L, S) tensor")
+    if out is None:
+        out = torch.empty((N, Hq, L, Ev), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((N, Hq, L), dtype=torch.float32, device=q.device)
+    if tuple(out.shape) != (N, Hq, L, Ev) or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("out has the wrong shape/dtype")
+    if tuple(lse.shape) != (N, Hq, L) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse has the wrong shape/dtype")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = load_library().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), N, Hq, H, L, S, E, Ev,
+                                     float(scale), MODES[mode], _ptr(sink), MASKS[mask_kind], int(window),
+                                     _ptr(bias), DTYPES[q.dtype], ctypes.c_void_p(stream.cuda_stream))
+    _check(st)
+    return out, lse
+
+
+def device_status(stream: torch.cuda.Stream | None = None) -> int:
+    """Synchronises the stream and returns (and clears) the kernels' fault status."""
+    s = stream or torch.cuda.current_stream()
+    return load_library().attn_device_status(ctypes.c_void_p(s.cuda_stream))
+
+
+def release_workspace():
+    load_library().attn_release_workspace()
+
+
+def version() -> int:
+    return load_library().attn_version()

@@ -1,0 +1,485 @@
+// bf16 attention forward for short query blocks (decode): split over keys.
+//
+// With L = 1 the whole batch holds only N*H independent (batch, KV head)
+// units of (Hq/H)*L query rows each, far too few to fill 148 SMs, and every
+// key/value byte is read exactly once, so the pass is bound by HBM bandwidth.
+// The key axis of every unit is cut into 64-key chunks and the N*H*chunks
+// work list is split evenly across a persistent grid (one CTA per SM): CTA b
+// takes chunks [b*T/G, (b+1)*T/G), which may span the end of one unit and the
+// start of the next.  For each unit segment it writes a partial
+// (m, l, acc[Ev]) per query row; the combine kernel merges the partials of
+// each unit and adds the sink logit (page "Attention Sink" §4.2: the sink
+// joins the denominator only).
+//
+// Per CTA: one TMA producer warp streams K and V chunks (3-D tensor maps,
+// 128-byte swizzle, zero fill past S) through a ring of stages; four consumer
+// warps each take 16 keys of every chunk.  The query rows of a unit (the
+// Hq/H heads of the KV group times L positions, at most 16) form the M = 16
+// side of mma.sync m16n8k16 products: S = Q K^T, then O += P V with P kept
+// in registers.  Each warp keeps its own online-softmax state; the four are
+// merged through shared memory at the end of a segment.
+//
+// Masks follow the bottom-right alignment of page "SDPA란 무엇인가" §4
+// (trap 3): query i of L sits at key position i + S - L.
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "ptx_sm100.cuh"
+
+namespace attn {
+
+namespace {
+
+constexpr int DC = 64;             // keys per chunk
+constexpr int DWARPS = 4;          // consumer warps (16 keys each)
+constexpr int DTHREADS = (DWARPS + 1) * 32;
+constexpr float D_RESCALE_THRESHOLD = 8.0f;
+
+struct DecodeParams {
+  const __nv_bfloat16* q;
+  __nv_bfloat16* out;
+  float* lse;
+  const float* sink;
+  const float* bias;
+  float* ws_acc;    // [slots][16][Ev]
+  float* ws_ml;     // [slots][16][2]
+  int N, Hq, H, L, S, group, R;
+  int mask_kind, window;
+  int kb_lo;        // first visible 64-key chunk (shared by all units)
+  int nc;           // chunks per unit
+  long long T;      // total chunks = N*H*nc
+  int G;            // persistent CTAs
+  int max_segs;     // partial slots per CTA
+  float c_dot;      // scale * log2e
+};
+
+template <int E, int EV>
+struct DCfg {
+  static constexpr int STAGE_BYTES = DC * (E + EV) * 2;
+  static constexpr int NSTAGE = (E + EV >= 256) ? 5 : 8;
+  static constexpr int OFF_STAGES = 0;
+  static constexpr int OFF_MERGE = NSTAGE * STAGE_BYTES;              // [DWARPS][16][EV] f32
+  static constexpr int OFF_ML = OFF_MERGE + DWARPS * 16 * EV * 4;     // [DWARPS][16][2] f32
+  static constexpr int OFF_BAR = OFF_ML + DWARPS * 16 * 2 * 4;
+  static constexpr int OFF_MISC = OFF_BAR + 2 * NSTAGE * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ long long seg_start(long long b, long long T, int G) { return (b * T) / G; }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(DWARPS * 32) : "memory"); }
+
+// byte offset of (row, 16-byte chunk c) inside a swizzled chunk buffer of 64-row, 128-byte boxes
+__device__ __forceinline__ uint32_t sw_off(int row, int c16) {
+  return (c16 >> 3) * (DC * 128) + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
+}
+
+template <int E, int EV>
+__global__ void __launch_bounds__(DTHREADS, 1)
+    decode_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          const DecodeParams p) {
+  using C = DCfg<E, EV>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sb = (raw_addr + 1023u) & ~1023u;
+  uint8_t* sp = smem_raw + (sb - raw_addr);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + C::OFF_MISC);
+  auto full_bar = [&](int s) -> uint32_t { return sb + C::OFF_BAR + 8u * s; };
+  auto empty_bar = [&](int s) -> uint32_t { return sb + C::OFF_BAR + 8u * (C::NSTAGE + s); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long c_begin = seg_start(blockIdx.x, p.T, p.G);
+  const long long c_end = seg_start(blockIdx.x + 1, p.T, p.G);
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), DWARPS);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (c_end <= c_begin) return;
+
+  if (warp == DWARPS) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int last_phase[C::NSTAGE];
+      for (int s = 0; s < C::NSTAGE; ++s) last_phase[s] = -1;
+      for (long long c = c_begin; c < c_end; ++c) {
+        const int idx = static_cast<int>(c - c_begin);
+        const int s = idx % C::NSTAGE;
+        const uint32_t ph = (idx / C::NSTAGE) & 1;
+        bool ok = mbar_wait(empty_bar(s), ph ^ 1);
+        if (!ok || *abort_flag) {
+          *abort_flag = 1;
+          break;
+        }
+        const long long u = c / p.nc;
+        const int key0 = (p.kb_lo + static_cast<int>(c % p.nc)) * DC;
+        const uint32_t dst = sb + C::OFF_STAGES + s * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(full_bar(s), C::STAGE_BYTES);
+        for (int b = 0; b < E / 64; ++b)
+          tma_load_3d(dst + b * (DC * 128), &tm_k, full_bar(s), b * 64, key0, static_cast<int>(u));
+        for (int b = 0; b < EV / 64; ++b)
+          tma_load_3d(dst + E * DC * 2 + b * (DC * 128), &tm_v, full_bar(s), b * 64, key0, static_cast<int>(u));
+        last_phase[s] = ph;
+      }
+      for (int s = 0; s < C::NSTAGE; ++s)
+        if (last_phase[s] >= 0) mbar_wait(full_bar(s), last_phase[s]);
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int rA = lane >> 2;       // fragment rows rA and rA + 8
+  const int cq = (lane & 3) * 2;  // fragment column pair
+  const int off = p.S - p.L;
+  int lo_r[2], hi_r[2];
+  bool live_r[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int r = rA + 8 * h;
+    live_r[h] = r < p.R;
+    const int i = live_r[h] ? (r % p.L) : 0;
+    lo_r[h] = (p.mask_kind == MASK_WINDOW) ? i + off - p.window + 1 : 0;
+    hi_r[h] = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, i + off + 1);
+  }
+
+  uint32_t qa[E / 16][4];
+  float o[EV / 8][4];
+  float m_run[2], l_run[2];
+  long long cur_unit = -1;
+  int seg = 0;
+  bool ok = true;
+
+  auto load_q = [&](long long u) {
+    const int n = static_cast<int>(u / p.H);
+    const int kvh = static_cast<int>(u % p.H);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = rA + 8 * h;
+      const __nv_bfloat16* qrow = nullptr;
+      if (r < p.R) {
+        const int hq = kvh * p.group + r / p.L;
+        const int i = r % p.L;
+        qrow = p.q + ((static_cast<size_t>(n) * p.Hq + hq) * p.L + i) * E;
+      }
+#pragma unroll
+      for (int kk = 0; kk < E / 16; ++kk) {
+        uint32_t lo = 0, hi = 0;
+        if (qrow) {
+          lo = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + cq);
+          hi = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + cq);
+        }
+        qa[kk][h] = lo;       // a0 (row rA) / a1 (row rA+8)
+        qa[kk][2 + h] = hi;   // a2 / a3
+      }
+    }
+  };
+  auto reset_state = [&]() {
+#pragma unroll
+    for (int t = 0; t < EV / 8; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+    m_run[0] = m_run[1] = -INFINITY;
+    l_run[0] = l_run[1] = 0.f;
+  };
+  float* merge_o = reinterpret_cast<float*>(sp + C::OFF_MERGE);
+  float* merge_ml = reinterpret_cast<float*>(sp + C::OFF_ML);
+  auto flush = [&](long long u, int segi) {
+    // per-warp state -> shared memory
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float l = l_run[h];
+      l += __shfl_xor_sync(0xffffffffu, l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      const int r = rA + 8 * h;
+      if ((lane & 3) == 0) {
+        merge_ml[(warp * 16 + r) * 2 + 0] = m_run[h];
+        merge_ml[(warp * 16 + r) * 2 + 1] = l;
+      }
+#pragma unroll
+      for (int t = 0; t < EV / 8; ++t) {
+        merge_o[(warp * 16 + r) * EV + t * 8 + cq] = o[t][2 * h];
+        merge_o[(warp * 16 + r) * EV + t * 8 + cq + 1] = o[t][2 * h + 1];
+      }
+    }
+    consumer_bar();
+    const size_t slot = static_cast<size_t>(blockIdx.x) * p.max_segs + segi;
+    for (int x = threadIdx.x; x < p.R * EV; x += DWARPS * 32) {
+      const int r = x / EV, e = x % EV;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < DWARPS; ++w) M = fmaxf(M, merge_ml[(w * 16 + r) * 2]);
+      float acc = 0.f, l = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < DWARPS; ++w) {
+          const float a = ex2(merge_ml[(w * 16 + r) * 2] - M);
+          acc = fmaf(a, merge_o[(w * 16 + r) * EV + e], acc);
+          l = fmaf(a, merge_ml[(w * 16 + r) * 2 + 1], l);
+        }
+      }
+      p.ws_acc[(slot * 16 + r) * EV + e] = acc;
+      if (e == 0) {
+        p.ws_ml[(slot * 16 + r) * 2 + 0] = M;
+        p.ws_ml[(slot * 16 + r) * 2 + 1] = l;
+      }
+    }
+    consumer_bar();
+  };
+
+  for (long long c = c_begin; c < c_end; ++c) {
+    const long long u = c / p.nc;
+    if (u != cur_unit) {
+      if (cur_unit >= 0) flush(cur_unit, seg++);
+      cur_unit = u;
+      load_q(u);
+      reset_state();
+    }
+    const int idx = static_cast<int>(c - c_begin);
+    const int s = idx % C::NSTAGE;
+    const bool w_ok = mbar_wait(full_bar(s), (idx / C::NSTAGE) & 1);
+    if (!__all_sync(0xffffffffu, w_ok)) {
+      *abort_flag = 1;
+      ok = false;
+      break;
+    }
+    const uint32_t kbuf = sb + C::OFF_STAGES + s * C::STAGE_BYTES;
+    const uint32_t vbuf = kbuf + E * DC * 2;
+    const int j0 = warp * 16;  // this warp's keys within the chunk
+    const int key0 = (p.kb_lo + static_cast<int>(c % p.nc)) * DC + j0;
+
+    // S = Q K^T for 16 keys (two n-tiles of 8)
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    {
+      const int mat = lane >> 3;
+      const int krow = j0 + (mat >> 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int kk = 0; kk < E / 16; ++kk) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kbuf + sw_off(krow, kk * 2 + (mat & 1)), b0, b1, b2, b3);
+        mma16816(sc[0], qa[kk], b0, b1);
+        mma16816(sc[1], qa[kk], b2, b3);
+      }
+    }
+    // logits in base 2, masks and bias
+    const bool need_mask = p.mask_kind != MASK_NONE || p.bias != nullptr || key0 + 16 > p.S;
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int h = e >> 1;
+        float zz = sc[t][e] * p.c_dot;
+        if (need_mask) {
+          const int key = key0 + t * 8 + cq + (e & 1);
+          if (key < lo_r[h] || key >= hi_r[h]) zz = -INFINITY;
+          if (p.bias != nullptr && live_r[h] && key < p.S)
+            zz = fmaf(p.bias[static_cast<size_t>((rA + 8 * h) % p.L) * p.S + key], LOG2E, zz);
+        }
+        sc[t][e] = zz;
+      }
+    // online softmax (lazy rescale)
+    float pr[2][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float mt = fmaxf(fmaxf(sc[0][2 * h], sc[0][2 * h + 1]), fmaxf(sc[1][2 * h], sc[1][2 * h + 1]));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+      const float m_new = fmaxf(m_run[h], mt);
+      if (m_new > m_run[h] + D_RESCALE_THRESHOLD) {
+        const float alpha = ex2(m_run[h] - m_new);
+        l_run[h] *= alpha;
+#pragma unroll
+        for (int t = 0; t < EV / 8; ++t) {
+          o[t][2 * h] *= alpha;
+          o[t][2 * h + 1] *= alpha;
+        }
+        m_run[h] = m_new;
+      }
+      const float mu = (m_run[h] == -INFINITY) ? 0.f : m_run[h];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        pr[t][2 * h] = ex2(sc[t][2 * h] - mu);
+        pr[t][2 * h + 1] = ex2(sc[t][2 * h + 1] - mu);
+        l_run[h] += pr[t][2 * h] + pr[t][2 * h + 1];
+      }
+    }
+    uint32_t pa[4];
+    pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+    pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+    pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+    pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+    // O += P V
+    {
+      const int mat = lane >> 3;
+      const int vrow = j0 + (mat & 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int t = 0; t < EV / 8; t += 2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vbuf + sw_off(vrow, t + (mat >> 1)), b0, b1, b2, b3);
+        mma16816(o[t], pa, b0, b1);
+        mma16816(o[t + 1], pa, b2, b3);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar(s));
+  }
+  ok = __all_sync(0xffffffffu, ok);
+  // all four consumer warps always reach this point together (same chunk list)
+  if (ok && cur_unit >= 0) flush(cur_unit, seg);
+}
+
+template <int EV>
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
+  const int u = blockIdx.x;
+  const int n = u / p.H, kvh = u % p.H;
+  const long long c_first = static_cast<long long>(u) * p.nc;
+  const long long c_last = c_first + p.nc - 1;
+  auto cta_of = [&](long long c) -> long long {
+    long long b = (c * p.G) / p.T;
+    while (b + 1 < p.G && seg_start(b + 1, p.T, p.G) <= c) ++b;
+    while (b > 0 && seg_start(b, p.T, p.G) > c) --b;
+    return b;
+  };
+  const long long b0 = cta_of(c_first), b1 = cta_of(c_last);
+  for (int x = threadIdx.x; x < p.R * EV; x += blockDim.x) {
+    const int r = x / EV, e = x % EV;
+    const int hq = kvh * p.group + r / p.L;
+    const int i = r % p.L;
+    const float s2 = p.sink ? p.sink[hq] * LOG2E : -INFINITY;
+    float M = s2;
+    for (long long b = b0; b <= b1; ++b) {
+      const long long segi = u - seg_start(b, p.T, p.G) / p.nc;
+      const size_t slot = static_cast<size_t>(b) * p.max_segs + segi;
+      M = fmaxf(M, p.ws_ml[(slot * 16 + r) * 2]);
+    }
+    float acc = 0.f, l = 0.f;
+    if (M != -INFINITY) {
+      for (long long b = b0; b <= b1; ++b) {
+        const long long segi = u - seg_start(b, p.T, p.G) / p.nc;
+        const size_t slot = static_cast<size_t>(b) * p.max_segs + segi;
+        const float a = ex2(p.ws_ml[(slot * 16 + r) * 2] - M);
+        acc = fmaf(a, p.ws_acc[(slot * 16 + r) * EV + e], acc);
+        l = fmaf(a, p.ws_ml[(slot * 16 + r) * 2 + 1], l);
+      }
+      l += ex2(s2 - M);
+    }
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    const size_t orow = (static_cast<size_t>(n) * p.Hq + hq) * p.L + i;
+    p.out[orow * EV + e] = __float2bfloat16_rn(acc * inv);
+    if (e == 0 && p.lse) p.lse[orow] = (l > 0.f) ? (M + __log2f(l)) * LN2 : -INFINITY;
+  }
+}
+
+struct DecodePlan {
+  int kb_lo, nc, G, max_segs;
+  long long T;
+};
+
+DecodePlan plan(const AttnArgs& a, int num_sms) {
+  DecodePlan d{};
+  const int off = a.S - a.L;
+  int lo = 0, hi = a.S;
+  if (a.mask_kind == MASK_CAUSAL || a.mask_kind == MASK_WINDOW) hi = a.S < off + a.L ? a.S : off + a.L;
+  if (a.mask_kind == MASK_WINDOW) lo = off - a.window + 1 > 0 ? off - a.window + 1 : 0;
+  if (hi < 1) hi = 1;  // keep one chunk so every row gets a (fully masked) partial
+  if (lo >= hi) lo = hi - 1;
+  d.kb_lo = lo / DC;
+  const int kb_hi = (hi + DC - 1) / DC;
+  d.nc = kb_hi - d.kb_lo;
+  d.T = static_cast<long long>(a.N) * a.H * d.nc;
+  d.G = static_cast<int>(d.T < num_sms ? d.T : num_sms);
+  const long long per = (d.T + d.G - 1) / d.G;
+  d.max_segs = static_cast<int>((per + d.nc - 1) / d.nc + 1);
+  return d;
+}
+
+template <int E, int EV>
+int launch_decode_impl(const AttnArgs& a, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream) {
+  using C = DCfg<E, EV>;
+  const DecodePlan d = plan(a, num_sms);
+  const size_t slots = static_cast<size_t>(d.G) * d.max_segs;
+  const size_t need = slots * 16 * (EV + 2) * sizeof(float);
+  if (ws_bytes < need) return -12;
+  CUtensorMap tk, tv;
+  if (!make_map_rows(&tk, a.k, E, a.S, static_cast<long long>(a.N) * a.H, DC)) return -13;
+  if (!make_map_rows(&tv, a.v, EV, a.S, static_cast<long long>(a.N) * a.H, DC)) return -13;
+  DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  p.sink = a.sink;
+  p.bias = a.bias;
+  p.ws_acc = static_cast<float*>(ws);
+  p.ws_ml = p.ws_acc + slots * 16 * EV;
+  p.N = a.N;
+  p.Hq = a.Hq;
+  p.H = a.H;
+  p.L = a.L;
+  p.S = a.S;
+  p.group = a.Hq / a.H;
+  p.R = p.group * a.L;
+  p.mask_kind = a.mask_kind;
+  p.window = a.window;
+  p.kb_lo = d.kb_lo;
+  p.nc = d.nc;
+  p.T = d.T;
+  p.G = d.G;
+  p.max_segs = d.max_segs;
+  p.c_dot = a.scale * LOG2E;
+  auto kern = decode_partial_kernel<E, EV>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return -13;
+  kern<<<d.G, DTHREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return -13;
+  decode_combine_kernel<EV><<<a.N * a.H, 128, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -13;
+}
+
+}  // namespace
+
+unsigned int take_status_decode(cudaStream_t s) { return take_device_status_local(s); }
+
+bool decode_eligible(const AttnArgs& a) { return (a.Hq / a.H) * a.L <= 16 && !a.rbf; }
+
+size_t decode_workspace_bytes(const AttnArgs& a, int num_sms) {
+  const DecodePlan d = plan(a, num_sms);
+  return static_cast<size_t>(d.G) * d.max_segs * 16 * (a.Ev + 2) * sizeof(float);
+}
+
+int launch_decode_bf16(const AttnArgs& a, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream) {
+  if (a.E == 128 && a.Ev == 128) return launch_decode_impl<128, 128>(a, ws, ws_bytes, num_sms, stream);
+  if (a.E == 64 && a.Ev == 64) return launch_decode_impl<64, 64>(a, ws, ws_bytes, num_sms, stream);
+  if (a.E == 64 && a.Ev == 128) return launch_decode_impl<64, 128>(a, ws, ws_bytes, num_sms, stream);
+  if (a.E == 128 && a.Ev == 64) return launch_decode_impl<128, 64>(a, ws, ws_bytes, num_sms, stream);
+  return -4;
+}
+
+}  // namespace attn

@@ -1,0 +1,51 @@
+// Internal launch interface shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cuda_runtime.h>
+
+namespace attn {
+
+enum MaskKind { MASK_NONE = 0, MASK_CAUSAL = 1, MASK_WINDOW = 2 };
+
+// Validated arguments of one forward call (see include/attn_b200.h).
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;          // nullable
+  int N, Hq, H, L, S, E, Ev;
+  float scale;
+  bool rbf;
+  const float* sink;   // [Hq] or nullptr
+  int mask_kind;
+  int window;
+  const float* bias;   // [L, S] or nullptr
+};
+
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+// Each launcher returns 0 or a negative attn_status code.
+int launch_prefill_bf16(const AttnArgs& a, cudaStream_t stream);
+int launch_fp32(const AttnArgs& a, cudaStream_t stream);
+
+// Decode (bf16, (Hq/H) * L <= 16): key-split partial kernel + combine kernel.
+bool decode_eligible(const AttnArgs& a);
+size_t decode_workspace_bytes(const AttnArgs& a, int num_sms);
+int launch_decode_bf16(const AttnArgs& a, void* workspace, size_t workspace_bytes, int num_sms,
+                       cudaStream_t stream);
+
+// Resolves cuTensorMapEncodeTiled through the runtime (no libcuda link).
+void* tensor_map_encoder();
+
+// bf16 [heads, rows, dim] tensor map with a 64 x box_rows x 1 box, 128-byte
+// swizzle and zero fill outside the tensor (defined in attn_abi.cu).
+bool make_map_rows(void* map, const void* base, int dim, long long rows, long long heads, int box_rows);
+
+// Read-and-clear of each kernel file's device fault word (synchronises `s`).
+unsigned int take_status_prefill(cudaStream_t s);
+unsigned int take_status_decode(cudaStream_t s);
+
+}  // namespace attn

@@ -1,0 +1,645 @@
+// bf16 fused attention forward (prefill) for sm_100a.
+//
+// One CTA owns two 128-row query tiles that share their key/value stream:
+// either two query heads of the same KV group at the same rows (GQA with an
+// even group size) or two consecutive row blocks of one head.  Warp roles:
+//
+//   warps 0-3   softmax for tile 0   (one thread per query row / TMEM lane)
+//   warps 4-7   softmax for tile 1
+//   warp  8     TMA producer: Q tiles once, then K and V tiles through rings
+//   warp  9     tcgen05 issuer: S_t = Q_t K^T into TMEM, O_t += P_t V from TMEM
+//   warp 10     key-norm warp (RBF only): ||k_j||^2 of each key tile from smem
+//
+// Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 and O_1 after
+// them.  P_t (bf16, two per column) overwrites the first 64 columns of S_t.
+//
+// Per key tile, softmax t reads its S_t row, forms the base-2 logit
+//   dot: z = s * scale*log2e            rbf: z = s * 2*scale*log2e - scale*log2e*||k||^2
+// adds mask / bias, updates the running max (the O rescale is skipped unless
+// the max grows by more than 2^8, which is exact because the final
+// normalisation uses the same stale max), writes P = 2^(z - m) and signals
+// the issuer.  The sink logit only enters the final normaliser.
+//
+// Method: page "Dot-Product Attention을 거리 기반 RBF-Attention으로 교체한 실험기"
+// (fused key-norm penalty in a tiled kernel), page "어텐션 메커니즘" §6 (tiling
+// with an online softmax), page "Attention Sink" §4.2 (sink in the denominator).
+
+#include <cfloat>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "ptx_sm100.cuh"
+
+namespace attn {
+
+namespace {
+
+constexpr int BM = 128;  // query rows per tile
+constexpr int BN = 128;  // keys per tile
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+
+struct PrefillParams {
+  __nv_bfloat16* out;
+  float* lse;
+  const float* sink;
+  const float* bias;
+  int N, Hq, H, L, S;
+  int group;        // Hq / H
+  int head_pairs;   // 1: tiles are (hq, hq+1) at the same rows; 0: (hq, rb), (hq, rb+1)
+  int n_rb;         // ceil(L / BM)
+  int n_items;
+  int mask_kind, window;
+  float c_dot;      // scale * log2e           (dot)
+  float c_rbf;      // 2 * scale * log2e       (rbf)
+  float c_kn;       // scale * log2e           (rbf key-norm penalty)
+};
+
+template <int E, int EV, bool RBF>
+struct Cfg {
+  static constexpr int NK = (E == 128) ? 2 : 4;
+  static constexpr int NV = (EV == 128) ? 2 : 4;
+  static constexpr int NKN = 4;
+  static constexpr int Q_BYTES = BM * E * 2;
+  static constexpr int K_BYTES = BN * E * 2;
+  static constexpr int V_BYTES = BN * EV * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NK * K_BYTES;
+  static constexpr int OFF_KN = OFF_V + NV * V_BYTES;
+  static constexpr int OFF_BAR = OFF_KN + (RBF ? NKN * BN * 4 : 0);
+  // barrier indices
+  static constexpr int B_Q = 0;
+  static constexpr int B_KFULL = 1;
+  static constexpr int B_KEMPTY = B_KFULL + NK;
+  static constexpr int B_VFULL = B_KEMPTY + NK;
+  static constexpr int B_VEMPTY = B_VFULL + NV;
+  static constexpr int B_SFULL = B_VEMPTY + NV;
+  static constexpr int B_PFULL = B_SFULL + 2;
+  static constexpr int B_OFULL = B_PFULL + 2;
+  static constexpr int B_KNFULL = B_OFULL + 2;
+  static constexpr int B_KNEMPTY = B_KNFULL + NKN;
+  static constexpr int B_DRAIN = B_KNEMPTY + NKN;
+  static constexpr int NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + base alignment slack
+  static constexpr int NUM_WARPS = RBF ? 11 : 10;
+  static constexpr int THREADS = NUM_WARPS * 32;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, EV, 1);
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct TileInfo {
+  int active;  // has query rows
+  int hq;
+  int r0;      // first query row
+  int jb_lo, jb_hi;  // key-tile range [jb_lo, jb_hi)
+};
+
+__device__ __forceinline__ void tile_range(const PrefillParams& p, TileInfo& t) {
+  t.jb_lo = t.jb_hi = 0;
+  if (!t.active) return;
+  const int off = p.S - p.L;
+  const int r_last = min(t.r0 + BM - 1, p.L - 1);
+  const int hi = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, r_last + off + 1);
+  const int lo = (p.mask_kind == MASK_WINDOW) ? max(0, t.r0 + off - p.window + 1) : 0;
+  if (hi <= lo) return;
+  t.jb_lo = lo / BN;
+  t.jb_hi = (hi + BN - 1) / BN;
+}
+
+__device__ __forceinline__ bool in_range(const TileInfo& t, int jb) { return jb >= t.jb_lo && jb < t.jb_hi; }
+
+// Bounded wait that also gives up as soon as another warp of the CTA has aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+      record_timeout();
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+template <int E, int EV, bool RBF>
+__global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+  using C = Cfg<E, EV, RBF>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sb = (raw_addr + 1023u) & ~1023u;
+  uint8_t* sp = smem_raw + (sb - raw_addr);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + C::OFF_MISC);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + C::OFF_MISC + 4);
+  auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8u * i; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item --------------------------------------------------------
+  int n, kvh;
+  TileInfo tile[2];
+  {
+    const int item = blockIdx.x;
+    if (p.head_pairs) {
+      const int hp_per = p.group / 2;
+      const int per_rb = p.N * p.H * hp_per;
+      const int rb = p.n_rb - 1 - item / per_rb;  // heavy (late) row blocks first
+      const int r = item % per_rb;
+      n = r / (p.H * hp_per);
+      const int rem = r % (p.H * hp_per);
+      kvh = rem / hp_per;
+      const int hq0 = kvh * p.group + 2 * (rem % hp_per);
+      tile[0] = {1, hq0, rb * BM, 0, 0};
+      tile[1] = {1, hq0 + 1, rb * BM, 0, 0};
+    } else {
+      const int n_rp = (p.n_rb + 1) / 2;
+      const int per_rp = p.N * p.Hq;
+      const int rp = n_rp - 1 - item / per_rp;
+      const int r = item % per_rp;
+      n = r / p.Hq;
+      const int hq = r % p.Hq;
+      kvh = hq / p.group;
+      tile[0] = {1, hq, 2 * rp * BM, 0, 0};
+      tile[1] = {(2 * rp + 1) * BM < p.L ? 1 : 0, hq, (2 * rp + 1) * BM, 0, 0};
+    }
+    tile_range(p, tile[0]);
+    tile_range(p, tile[1]);
+  }
+  const bool has0 = tile[0].jb_hi > tile[0].jb_lo;
+  const bool has1 = tile[1].jb_hi > tile[1].jb_lo;
+  int u_lo = 0, u_hi = 0;
+  if (has0 && has1) {
+    u_lo = min(tile[0].jb_lo, tile[1].jb_lo);
+    u_hi = max(tile[0].jb_hi, tile[1].jb_hi);
+  } else if (has0) {
+    u_lo = tile[0].jb_lo;
+    u_hi = tile[0].jb_hi;
+  } else if (has1) {
+    u_lo = tile[1].jb_lo;
+    u_hi = tile[1].jb_hi;
+  }
+
+  // ---- setup ------------------------------------------------------------
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(C::B_Q), 1);
+    for (int s = 0; s < C::NK; ++s) {
+      mbar_init(bar(C::B_KFULL + s), 1);
+      mbar_init(bar(C::B_KEMPTY + s), RBF ? 2 : 1);
+    }
+    for (int s = 0; s < C::NV; ++s) {
+      mbar_init(bar(C::B_VFULL + s), 1);
+      mbar_init(bar(C::B_VEMPTY + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(C::B_SFULL + t), 1);
+      mbar_init(bar(C::B_PFULL + t), 128);
+      mbar_init(bar(C::B_OFULL + t), 1);
+    }
+    for (int s = 0; s < C::NKN; ++s) {
+      mbar_init(bar(C::B_KNFULL + s), 32);
+      mbar_init(bar(C::B_KNEMPTY + s), 256);
+    }
+    mbar_init(bar(C::B_DRAIN), 1);
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      uint32_t qbytes = (has0 ? C::Q_BYTES : 0) + (has1 ? C::Q_BYTES : 0);
+      if (qbytes) {
+        mbar_arrive_expect_tx(bar(C::B_Q), qbytes);
+        for (int t = 0; t < 2; ++t) {
+          if (!(t == 0 ? has0 : has1)) continue;
+          for (int b = 0; b < E / 64; ++b)
+            tma_load_3d(sb + C::OFF_Q + t * C::Q_BYTES + b * (BM * 128), &tm_q, bar(C::B_Q), b * 64,
+                        tile[t].r0, n * p.Hq + tile[t].hq);
+        }
+      }
+      int last_k_phase[C::NK], last_v_phase[C::NV];
+      for (int s = 0; s < C::NK; ++s) last_k_phase[s] = -1;
+      for (int s = 0; s < C::NV; ++s) last_v_phase[s] = -1;
+      for (int jb = u_lo; jb < u_hi; ++jb) {
+        const int idx = jb - u_lo;
+        const int ks = idx % C::NK;
+        const uint32_t kph = (idx / C::NK) & 1;
+        if (!wait_bar(bar(C::B_KEMPTY + ks), kph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::B_KFULL + ks), C::K_BYTES);
+        for (int b = 0; b < E / 64; ++b)
+          tma_load_3d(sb + C::OFF_K + ks * C::K_BYTES + b * (BN * 128), &tm_k, bar(C::B_KFULL + ks), b * 64,
+                      jb * BN, n * p.H + kvh);
+        last_k_phase[ks] = kph;
+        const int vs = idx % C::NV;
+        const uint32_t vph = (idx / C::NV) & 1;
+        if (!wait_bar(bar(C::B_VEMPTY + vs), vph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::B_VFULL + vs), C::V_BYTES);
+        for (int b = 0; b < EV / 64; ++b)
+          tma_load_3d(sb + C::OFF_V + vs * C::V_BYTES + b * (BN * 128), &tm_v, bar(C::B_VFULL + vs), b * 64,
+                      jb * BN, n * p.H + kvh);
+        last_v_phase[vs] = vph;
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      if (qbytes) mbar_wait(bar(C::B_Q), 0);
+      for (int s = 0; s < C::NK; ++s)
+        if (last_k_phase[s] >= 0) mbar_wait(bar(C::B_KFULL + s), last_k_phase[s]);
+      for (int s = 0; s < C::NV; ++s)
+        if (last_v_phase[s] >= 0) mbar_wait(bar(C::B_VFULL + s), last_v_phase[s]);
+    }
+  } else if (warp == 9) {
+    // ================= tcgen05 issuer =================
+    if (lane == 0) {
+      bool ok = true;
+      if (u_hi > u_lo) ok = wait_bar(bar(C::B_Q), 0, abort_flag);
+      tc_fence_after();
+      int pend[2] = {-1, -1};
+      int pv_count[2] = {0, 0};
+      int v_waited = u_lo - 1;  // highest key tile whose V landing was awaited
+      int v_cur = -1, v_cur_uses = 0;
+
+      auto issue_pv = [&](int t, int jbp) -> bool {
+        const int idxp = jbp - u_lo;
+        const int vs = idxp % C::NV;
+        if (jbp > v_waited) {
+          if (!wait_bar(bar(C::B_VFULL + vs), (idxp / C::NV) & 1, abort_flag)) return false;
+          v_waited = jbp;
+        }
+        if (!wait_bar(bar(C::B_PFULL + t), pv_count[t] & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + 256 + t * EV;
+        const uint32_t a = tmem + t * 128;
+        const uint32_t vbase = sb + C::OFF_V + vs * C::V_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // B = V tile, MN-major: 16 keys per step = 16 rows of 128 B; second 64-column box at +BN*128
+          const uint64_t bdesc = smem_desc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
+          mma_ts(d, a + kk * 8, bdesc, C::IDESC_PV, (pv_count[t] > 0 || kk > 0) ? 1u : 0u);
+        }
+        pv_count[t]++;
+        const int uses = (in_range(tile[0], jbp) ? 1 : 0) + (in_range(tile[1], jbp) ? 1 : 0);
+        if (jbp != v_cur) {
+          v_cur = jbp;
+          v_cur_uses = 0;
+        }
+        if (++v_cur_uses == uses) mma_commit(bar(C::B_VEMPTY + vs));
+        return true;
+      };
+
+      for (int jb = u_lo; ok && jb < u_hi; ++jb) {
+        const int idx = jb - u_lo;
+        const int ks = idx % C::NK;
+        if (!wait_bar(bar(C::B_KFULL + ks), (idx / C::NK) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!in_range(tile[t], jb)) continue;
+          if (pend[t] >= 0) {
+            if (!issue_pv(t, pend[t])) {
+              ok = false;
+              break;
+            }
+          }
+          const uint32_t d = tmem + t * 128;
+          const uint32_t qbase = sb + C::OFF_Q + t * C::Q_BYTES;
+          const uint32_t kbase = sb + C::OFF_K + ks * C::K_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < E / 16; ++kk) {
+            const uint32_t koff = (kk / 4) * (BM * 128) + (kk % 4) * 32;
+            const uint64_t adesc = smem_desc_sw128(qbase + koff, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(kbase + koff, 16, 1024);
+            mma_ss(d, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(C::B_SFULL + t));
+          pend[t] = jb;
+        }
+        if (ok) mma_commit(bar(C::B_KEMPTY + ks));
+        if (ok && !in_range(tile[0], jb) && !in_range(tile[1], jb)) {
+          // a key tile neither query tile reads: let its V copy land, then free the slot
+          const int vs = idx % C::NV;
+          if (!wait_bar(bar(C::B_VFULL + vs), (idx / C::NV) & 1, abort_flag)) ok = false;
+          else mma_commit(bar(C::B_VEMPTY + vs));
+          if (jb > v_waited) v_waited = jb;
+        }
+      }
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (pend[t] < 0) continue;
+        if (!issue_pv(t, pend[t])) {
+          ok = false;
+          break;
+        }
+        mma_commit(bar(C::B_OFULL + t));
+      }
+      // drain: all issued tensor-core work completes before TMEM is released
+      mma_commit(bar(C::B_DRAIN));
+      mbar_wait(bar(C::B_DRAIN), 0);
+    }
+  } else if (RBF && warp == 10) {
+    // ================= key-norm warp (RBF) =================
+    for (int jb = u_lo; jb < u_hi; ++jb) {
+      const int idx = jb - u_lo;
+      const int ks = idx % C::NK;
+      const int slot = idx % C::NKN;
+      if (!wait_bar(bar(C::B_KFULL + ks), (idx / C::NK) & 1, abort_flag)) break;
+      if (!wait_bar(bar(C::B_KNEMPTY + slot), ((idx / C::NKN) & 1) ^ 1, abort_flag)) break;
+      const uint8_t* ktile = sp + C::OFF_K + ks * C::K_BYTES;
+      float* kn = reinterpret_cast<float*>(sp + C::OFF_KN) + slot * BN;
+#pragma unroll
+      for (int rr = 0; rr < BN / 32; ++rr) {
+        const int r = lane + 32 * rr;
+        float acc = 0.f;
+#pragma unroll
+        for (int b = 0; b < E / 64; ++b) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 w = *reinterpret_cast<const uint4*>(ktile + b * (BN * 128) + r * 128 + ((c ^ (r & 7)) << 4));
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float lo = __uint_as_float(ws[e] << 16);
+              const float hi = __uint_as_float(ws[e] & 0xFFFF0000u);
+              acc = fmaf(lo, lo, acc);
+              acc = fmaf(hi, hi, acc);
+            }
+          }
+        }
+        kn[r] = acc * p.c_kn;
+      }
+      __syncwarp();
+      mbar_arrive(bar(C::B_KNFULL + slot));
+      if (lane == 0) mbar_arrive(bar(C::B_KEMPTY + ks));
+    }
+  } else if (warp < 8) {
+    // ================= softmax warpgroups =================
+    const int t = warp >> 2;
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const TileInfo T = t ? tile[1] : tile[0];
+    const int i = T.r0 + row;
+    const int off = p.S - p.L;
+    const int lo_i = (p.mask_kind == MASK_WINDOW) ? (i + off - p.window + 1) : 0;
+    const int hi_i = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, i + off + 1);
+    const int first_row_hi = T.r0 + off + 1;               // key limit of the tile's first row
+    const int last_row_lo = min(T.r0 + BM - 1, p.L - 1) + off - p.window + 1;
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + t * 128;
+    const uint32_t t_o = tmem + lane_base + 256 + t * EV;
+    const bool has_bias = p.bias != nullptr;
+    const float* bias_row = has_bias && i < p.L ? p.bias + static_cast<size_t>(i) * p.S : nullptr;
+
+    float m_run = -INFINITY, l_run = 0.f;
+    int it = 0;
+    bool ok = true;
+    for (int jb = u_lo; jb < u_hi; ++jb) {
+      const int idx = jb - u_lo;
+      const int slot = idx % C::NKN;
+      if (RBF) {
+        const bool w = wait_bar(bar(C::B_KNFULL + slot), (idx / C::NKN) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+      }
+      if (!in_range(T, jb)) {
+        if (RBF) mbar_arrive(bar(C::B_KNEMPTY + slot));
+        continue;
+      }
+      {
+        const bool w = wait_bar(bar(C::B_SFULL + t), it & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+      }
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tmem_wait_ld();
+      float* z = reinterpret_cast<float*>(sr);
+
+      const int k0 = jb * BN;
+      const bool need_mask = ((k0 + BN) > p.S) ||
+                             (p.mask_kind != MASK_NONE && (k0 + BN) > first_row_hi) ||
+                             (p.mask_kind == MASK_WINDOW && k0 < last_row_lo);
+      const bool scaled = RBF || need_mask || has_bias;
+      if (RBF) {
+        const float* kn = reinterpret_cast<const float*>(sp + C::OFF_KN) + slot * BN;
+#pragma unroll
+        for (int c = 0; c < BN; c += 4) {
+          const float4 kv = *reinterpret_cast<const float4*>(kn + c);
+          z[c + 0] = fmaf(z[c + 0], p.c_rbf, -kv.x);
+          z[c + 1] = fmaf(z[c + 1], p.c_rbf, -kv.y);
+          z[c + 2] = fmaf(z[c + 2], p.c_rbf, -kv.z);
+          z[c + 3] = fmaf(z[c + 3], p.c_rbf, -kv.w);
+        }
+        __syncwarp();
+        mbar_arrive(bar(C::B_KNEMPTY + slot));
+      } else if (scaled) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) z[c] *= p.c_dot;
+      }
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          const int key = k0 + c;
+          if (key < lo_i || key >= hi_i) z[c] = -INFINITY;
+        }
+      }
+      if (has_bias && bias_row != nullptr) {
+#pragma unroll 8
+        for (int c = 0; c < BN; ++c) {
+          const int key = k0 + c;
+          if (key < p.S) z[c] = fmaf(__ldg(bias_row + key), LOG2E, z[c]);
+        }
+      }
+      float mt = z[0];
+#pragma unroll
+      for (int c = 1; c < BN; ++c) mt = fmaxf(mt, z[c]);
+      if (!scaled) mt *= p.c_dot;
+
+      const float m_new = fmaxf(m_run, mt);
+      const bool rescale = m_new > m_run + RESCALE_THRESHOLD;
+      if (__any_sync(0xffffffffu, rescale)) {
+        const float alpha = rescale ? ex2(m_run - m_new) : 1.f;
+        if (rescale) {
+          l_run *= alpha;
+          m_run = m_new;
+        }
+        if (it > 0) {
+#pragma unroll 1
+          for (int c = 0; c < EV; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(t_o + c, o);
+          }
+        }
+      }
+      const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+      float rs = 0.f;
+      uint32_t pk[64];
+      if (scaled) {
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float p0 = ex2(z[c] - mu);
+          const float p1 = ex2(z[c + 1] - mu);
+          rs += p0 + p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+      } else {
+        const float nm = -mu;
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float p0 = ex2(fmaf(z[c], p.c_dot, nm));
+          const float p1 = ex2(fmaf(z[c + 1], p.c_dot, nm));
+          rs += p0 + p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+      }
+      l_run += rs;
+      tmem_st32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PFULL + t));
+      ++it;
+    }
+
+    // ---- epilogue ----
+    ok = __all_sync(0xffffffffu, ok);
+    if (T.active && ok) {
+      bool have_o = it > 0;
+      if (have_o) {
+        have_o = __all_sync(0xffffffffu, wait_bar(bar(C::B_OFULL + t), 0, abort_flag));
+        tc_fence_after();
+      }
+      const float s2 = p.sink ? p.sink[T.hq] * LOG2E : -INFINITY;
+      const float M2 = fmaxf(m_run, s2);
+      float inv = 0.f, lse2 = -INFINITY;
+      if (M2 != -INFINITY) {
+        const float a = ex2(m_run - M2);
+        const float lp = l_run * a + ex2(s2 - M2);
+        if (lp > 0.f) {
+          inv = a / lp;
+          lse2 = M2 + __log2f(lp);
+        }
+      }
+      const bool row_ok = i < p.L;
+      const size_t orow = (static_cast<size_t>(n) * p.Hq + T.hq) * p.L + i;
+      __nv_bfloat16* op = p.out + orow * EV;
+#pragma unroll 1
+      for (int c = 0; c < EV; c += 32) {
+        uint32_t o[32];
+        if (have_o) {
+          tmem_ld32(t_o + c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        if (row_ok) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(op + c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+      if (row_ok && p.lse) p.lse[orow] = lse2 * LN2;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+template <int E, int EV, bool RBF>
+int launch_impl(const AttnArgs& a, cudaStream_t stream) {
+  using C = Cfg<E, EV, RBF>;
+  CUtensorMap tq, tk, tv;
+  if (!make_map_rows(&tq, a.q, E, a.L, static_cast<long long>(a.N) * a.Hq, BM)) return -13;
+  if (!make_map_rows(&tk, a.k, E, a.S, static_cast<long long>(a.N) * a.H, BN)) return -13;
+  if (!make_map_rows(&tv, a.v, EV, a.S, static_cast<long long>(a.N) * a.H, BN)) return -13;
+  PrefillParams p{};
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  p.sink = a.sink;
+  p.bias = a.bias;
+  p.N = a.N;
+  p.Hq = a.Hq;
+  p.H = a.H;
+  p.L = a.L;
+  p.S = a.S;
+  p.group = a.Hq / a.H;
+  p.head_pairs = (p.group % 2 == 0) ? 1 : 0;
+  p.n_rb = (a.L + BM - 1) / BM;
+  if (p.head_pairs)
+    p.n_items = p.N * p.H * (p.group / 2) * p.n_rb;
+  else
+    p.n_items = p.N * p.Hq * ((p.n_rb + 1) / 2);
+  p.mask_kind = a.mask_kind;
+  p.window = a.window;
+  p.c_dot = a.scale * LOG2E;
+  p.c_rbf = 2.f * a.scale * LOG2E;
+  p.c_kn = a.scale * LOG2E;
+  auto kern = prefill_kernel<E, EV, RBF>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return -13;
+  kern<<<p.n_items, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -13;
+}
+
+}  // namespace
+
+unsigned int take_status_prefill(cudaStream_t s) { return take_device_status_local(s); }
+
+int launch_prefill_bf16(const AttnArgs& a, cudaStream_t stream) {
+  const bool r = a.rbf;
+#define ATTN_PREFILL_CASE(e, ev)                                            \
+  if (a.E == e && a.Ev == ev) return r ? launch_impl<e, ev, true>(a, stream) \
+                                       : launch_impl<e, ev, false>(a, stream);
+  ATTN_PREFILL_CASE(64, 64)
+  ATTN_PREFILL_CASE(128, 128)
+  ATTN_PREFILL_CASE(64, 128)
+  ATTN_PREFILL_CASE(128, 64)
+#undef ATTN_PREFILL_CASE
+  return -4;
+}
+
+}  // namespace attn

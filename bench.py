@@ -1,0 +1,483 @@
+#!/usr/bin/env python
+"""Benchmark of the fused attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-extra]
+
+A step is one call of the library's attention forward (``attn_fwd``) over one
+batch of the workload, inputs resident in HBM.  Steps are timed with CUDA
+events on the launching stream; a 256 MiB buffer is rewritten between steps
+(outside the events) so every step starts with a cold L2.  Under torchrun each
+rank runs the same per-GPU workload (weak scaling, no collective on the data
+path); the barrier-bracketed timed region is reduced with MAX over ranks and
+rank 0 prints one JSON line.
+
+The default workload is the bf16 causal dot-product prefill (N=4, H=16,
+L=S=2048, E=Ev=128); its throughput in TFLOP/s (2*(E+Ev) FLOPs per visible
+query/key pair) is `value`.  The other reference workloads are measured too
+and reported under "workloads" (TFLOP/s for prefill, KV-read GB/s for decode).
+
+``--impl reference`` runs the reference arm: the float64 CPU oracle, timed on
+the host cores on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import workloads as sw  # noqa: E402
+
+METRIC = "attn fwd TFLOP/s (prefill), KV-read GB/s (decode), % of B200 roofline"
+DEFAULT_WORKLOAD = "dot_causal_2k_bf16"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch of the dominant kernel from an ncu capture of the same
+# kernel build (profiles/*.md records the command and counters); None until taken.
+NCU_TRAFFIC_BYTES = {}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+# ---------------------------------------------------------------------------
+
+def visible_pairs(r: sw.Recipe) -> int:
+    """Number of (query, key) pairs the mask leaves visible, per (n, hq)."""
+    i = np.arange(r.L, dtype=np.int64)
+    ip = i + (r.S - r.L)
+    if r.mask_kind == "none" or r.bias != "none":
+        hi = np.full(r.L, r.S, dtype=np.int64)
+        lo = np.zeros(r.L, dtype=np.int64)
+        if r.mask_kind != "none":
+            hi = np.minimum(r.S, ip + 1)
+            if r.mask_kind == "window":
+                lo = np.maximum(0, ip - r.window + 1)
+    else:
+        hi = np.minimum(r.S, ip + 1)
+        lo = np.maximum(0, ip - r.window + 1) if r.mask_kind == "window" else np.zeros(r.L, dtype=np.int64)
+    return int(np.maximum(0, hi - lo).sum())
+
+
+def is_decode(r: sw.Recipe) -> bool:
+    return r.dtype == "bf16" and r.mode == "dot" and (r.Hq // r.H) * r.L <= 16
+
+
+def work_units(r: sw.Recipe):
+    """(amount, unit, roofline bound) of one step of workload r on one GPU."""
+    if is_decode(r):
+        kv_bytes = r.N * r.H * r.S * (r.E + r.Ev) * 2
+        return kv_bytes, "GB/s", "hbm"
+    flops = 2 * (r.E + r.Ev) * visible_pairs(r) * r.N * r.Hq
+    return flops, "TFLOP/s", "tensor"
+
+
+def rate(amount: float, seconds: float, unit: str) -> float:
+    return amount / seconds / (1e12 if unit == "TFLOP/s" else 1e9)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks (NVML, read only)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        0x0000000000000008: "hw_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000004: "sw_power_cap",
+        0x0000000000000080: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001
+            self.nvml = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                mask = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.nvml is not None:
+            self.t.join()
+
+    def summary(self):
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    return world, rank, local, pg
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+def max_over_ranks(pg, value: float) -> float:
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_device(fn, steps, warmup, flush_buf, stream):
+    """Sum of per-step CUDA-event times (seconds); L2 flushed before every step."""
+    import torch
+    for _ in range(warmup):
+        flush_buf.fill_(1.0)
+        fn()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for k in range(steps):
+        flush_buf.fill_(float(k))
+        starts[k].record(stream)
+        fn()
+        ends[k].record(stream)
+    torch.cuda.synchronize()
+    return sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / 1e3
+
+
+def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=False):
+    import torch
+
+    import attention_tiled_attn_b200 as attn
+    from synth import gpu as sgpu
+
+    r = sw.RECIPES[name]
+    t = sgpu.generate_on_device(r)
+    out = torch.empty((r.N, r.Hq, r.L, r.Ev), dtype=t["q"].dtype, device="cuda")
+    lse = torch.empty((r.N, r.Hq, r.L), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=r.mode, sink=t["sink"], mask_kind=r.mask_kind,
+                      window=r.window, bias=t["bias"], out=out, lse=lse, stream=stream)
+
+    amount, unit, bound = work_units(r)
+    barrier(pg)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
+    if sampler:
+        sampler.__enter__()
+    secs = time_device(step, steps, warmup, flush_buf, stream)
+    if sampler:
+        sampler.__exit__()
+    torch.cuda.synchronize()
+    barrier(pg)
+    secs_max = max_over_ranks(pg, secs)
+    status = attn.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after {name}")
+    per_launch = secs / steps
+    achieved = rate(amount, per_launch, unit)
+    if bound == "tensor":
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        punit = "TFLOP/s"
+    else:
+        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        punit = "GB/s"
+    traffic = NCU_TRAFFIC_BYTES.get(name)
+    res = {
+        "recipe": r, "amount": amount, "unit": unit, "secs_max": secs_max, "secs": secs,
+        "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": punit,
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                     else "fallback"},
+        "launches_per_step": 2 if is_decode(r) else 1,
+        "clocks": sampler.summary() if sampler else None,
+        "tensors": t, "out": out, "lse": lse,
+    }
+    return res
+
+
+def e2e_measure(res, steps, warmup):
+    """Same metric through the public API with pinned host buffers: every step
+    copies its inputs host->device, runs attn_fwd and reads the output back."""
+    import torch
+
+    import attention_tiled_attn_b200 as attn
+    r = res["recipe"]
+    t = res["tensors"]
+    host = {k: t[k].cpu().pin_memory() for k in ("q", "k", "v")}
+    dev = {k: torch.empty_like(t[k]) for k in ("q", "k", "v")}
+    out_host = torch.empty(res["out"].shape, dtype=res["out"].dtype).pin_memory()
+    lse_host = torch.empty(res["lse"].shape, dtype=torch.float32).pin_memory()
+    stream = torch.cuda.current_stream()
+    h2d = sum(host[k].numel() * host[k].element_size() for k in host)
+    d2h = out_host.numel() * out_host.element_size() + lse_host.numel() * 4
+
+    def step():
+        for k in ("q", "k", "v"):
+            dev[k].copy_(host[k], non_blocking=True)
+        attn.attn_fwd(dev["q"], dev["k"], dev["v"], scale=r.scale, mode=r.mode, sink=t["sink"],
+                      mask_kind=r.mask_kind, window=r.window, bias=t["bias"], out=res["out"], lse=res["lse"],
+                      stream=stream)
+        out_host.copy_(res["out"], non_blocking=True)
+        lse_host.copy_(res["lse"], non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    secs = a.elapsed_time(b) / 1e3
+    for k in list(host):
+        del host[k]
+    return {"value": round(rate(res["amount"], secs / steps, res["unit"]), 3), "unit": res["unit"],
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}, secs
+
+
+def _oracle_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return int(max([i.get("num_threads", 1) for i in threadpool_info()] + [1]))
+    except Exception:  # noqa: BLE001
+        return int(os.cpu_count() or 1)
+
+
+class OracleSample:
+    """Runs the float64 oracle (as it stands) on row blocks of one (n, hq) head
+    of workload r, and converts the time into the workload's unit."""
+
+    def __init__(self, r: sw.Recipe, n: int = 0, hq: int = 0):
+        from oracle import attention as orc
+        self.orc, self.r, self.hq = orc, r, hq
+        kvh = hq // r.group
+        self.q = sw.tensor_slice_f64(r, "q", n, hq)
+        self.k = sw.tensor_slice_f64(r, "k", n, kvh)
+        self.v = sw.tensor_slice_f64(r, "v", n, kvh)
+        s = sw.sink_logits(r)
+        self.sink = None if s is None else float(s[hq])
+        self.bias = sw.bias_matrix(r)
+        amount, self.unit, _ = work_units(r)
+        self.per_pair = amount / (r.N * r.Hq * max(1, visible_pairs(r)))
+
+    def rows_amount(self, rows):
+        r = self.r
+        ip = rows + (r.S - r.L)
+        hi = np.full(rows.size, r.S) if r.mask_kind == "none" or r.bias != "none" else np.minimum(r.S, ip + 1)
+        if r.mask_kind != "none" and r.bias != "none":
+            hi = np.minimum(r.S, ip + 1)
+        lo = np.maximum(0, ip - r.window + 1) if r.mask_kind == "window" else np.zeros(rows.size)
+        return float(np.maximum(0, hi - lo).sum()) * self.per_pair
+
+    def run(self, rows):
+        r = self.r
+        for i0 in range(0, rows.size, 256):
+            rr = rows[i0:i0 + 256]
+            self.orc.attend_rows(self.q[rr], rr, self.k, self.v, r.L, scale=r.scale, mode=r.mode, sink=self.sink,
+                                 mask_kind=r.mask_kind, window=r.window,
+                                 bias_rows=None if self.bias is None else self.bias[rr])
+        return self.rows_amount(rows)
+
+
+def cpu_baseline(r: sw.Recipe, budget_s: float = 12.0):
+    """Oracle throughput on the host cores over a bounded sample (~budget_s of
+    compute): consecutive 256-row blocks of head (0, 0), from the last rows
+    (the heaviest under a causal mask) backwards."""
+    smp = OracleSample(r)
+    done, secs, blocks = 0.0, 0.0, 0
+    for i1 in range(r.L, 0, -256):
+        rows = np.arange(max(0, i1 - 256), i1)
+        t0 = time.perf_counter()
+        done += smp.run(rows)
+        secs += time.perf_counter() - t0
+        blocks += 1
+        if secs > budget_s:
+            break
+    return {"value": round(rate(done, secs, smp.unit), 6), "unit": smp.unit, "cores": _oracle_cores(),
+            "kind": "oracle",
+            "sample": f"{blocks} x 256-row blocks of head (n=0, hq=0) of {r.name} ({secs:.1f} s of float64 numpy)"}
+
+
+def ours(args):
+    import torch
+    world, rank, local, pg = dist_setup(args)
+    peaks, peak_kind = load_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    main = run_workload(args.workload, args.steps, args.warmup, pg, flush, peaks, peak_kind, clocks=True)
+    r = main["recipe"]
+    e2e, _ = e2e_measure(main, max(3, min(args.steps, 20)), 2)
+    extra = {}
+    if not args.no_extra:
+        for name in sw.RECIPES:
+            if name == args.workload or sw.RECIPES[name].dtype != "bf16":
+                continue
+            main_t = {k: main[k] for k in ("tensors", "out", "lse")}
+            res = run_workload(name, max(5, args.steps // 4), args.warmup, pg, flush, peaks, peak_kind)
+            rr = res["recipe"]
+            extra[name] = {
+                "value": round(rate(res["amount"] * world, res["secs_max"] / max(5, args.steps // 4),
+                                    res["unit"]), 2),
+                "unit": res["unit"], "ms_per_step": round(res["secs_max"] / max(5, args.steps // 4) * 1e3, 4),
+                "roofline_frac": res["roofline"]["frac"], "bound": res["roofline"]["bound"],
+                "mode": rr.mode, "sink": rr.sink != "none", "mask": rr.mask_kind,
+            }
+            del res
+            torch.cuda.empty_cache()
+    if rank == 0:
+        amount_all = main["amount"] * world
+        line = {
+            "metric": METRIC,
+            "value": round(rate(amount_all, main["secs_max"] / args.steps, main["unit"]), 3),
+            "unit": main["unit"],
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(main["secs_max"] / args.steps * 1e3, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if r.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded counter-based N(0,1) draws, see synth/workloads.py)",
+            "config": {"workload": r.name, "N": r.N, "Hq": r.Hq, "H": r.H, "L": r.L, "S": r.S, "E": r.E,
+                       "Ev": r.Ev, "mode": r.mode, "mask": r.mask_kind, "window": r.window,
+                       "sink": r.sink != "none", "scale": r.scale,
+                       "parallelism": f"replicas x{world} (independent batches, no collective)",
+                       "l2": "flushed: 256 MiB rewritten between timed steps, outside the events"},
+            "roofline": main["roofline"],
+            "cpu_baseline": cpu_baseline(r) if world == 1 else None,
+            "e2e": e2e,
+            "gpu_launches": main["launches_per_step"] * args.steps,
+            "clocks": main["clocks"],
+            "impl": "ours",
+            "workloads": extra,
+        }
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    r = sw.RECIPES[args.workload]
+    smp = OracleSample(r)
+    # calibrate the per-step sample so that warmup + steps take ~90 s in total
+    cal = np.arange(max(0, r.L - 64), r.L)
+    t0 = time.perf_counter()
+    smp.run(cal)
+    per_row = (time.perf_counter() - t0) / cal.size
+    rows_per_step = int(min(r.L, max(8, 90.0 / (args.steps + args.warmup) / max(per_row, 1e-9))))
+    rows = np.arange(r.L - rows_per_step, r.L)
+    for _ in range(args.warmup):
+        smp.run(rows)
+    done = 0.0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        done += smp.run(rows)
+    secs = time.perf_counter() - t0
+    value = rate(done, secs, smp.unit)
+    sample = f"last {rows_per_step} rows of head (n=0, hq=0) of {r.name} per step, float64 numpy oracle"
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": smp.unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": r.name, "N": r.N, "Hq": r.Hq, "H": r.H, "L": r.L, "S": r.S, "E": r.E,
+                   "Ev": r.Ev, "mode": r.mode, "mask": r.mask_kind},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 6), "unit": smp.unit, "cores": _oracle_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": smp.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(sw.RECIPES))
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        reference(args)
+    else:
+        ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,128 @@
+/*
+ * attn_b200.h -- C ABI of the fused attention forward for NVIDIA B200 (sm_100a).
+ *
+ * One operation:  out = softmax(z + B) V   per (batch n, query head hq, query row i),
+ * with the score z in one of two modes and an optional per-head sink logit.
+ *
+ *   dot   z_ij = scale * <q_i, k_j>
+ *         (page "어텐션 메커니즘" section 2, the softmax(QK^T/sqrt(d_k))V definition;
+ *          page "SDPA란 무엇인가" section 1, softmax(QK^T/sqrt(E) + B)V and its steps)
+ *   rbf   z_ij = -scale * ||q_i - k_j||^2, evaluated in the expanded frame
+ *         2*scale*<q_i,k_j> - scale*||k_j||^2 (the query norm cancels by softmax
+ *         shift invariance; the key-norm penalty is formed on chip from each key
+ *         tile).  (page "Dot-Product Attention을 거리 기반 RBF-Attention으로 교체한
+ *          실험기", 섹션별 상세: the squared-distance expansion and the fused kernel)
+ *   sink  a per-query-head logit s[hq] joins the softmax denominator but not the
+ *         value sum:  out_i = sum_j e^{z_ij} v_j / (e^{s} + sum_j e^{z_ij})
+ *         (page "Attention Sink" sections 4.2 and 5.2-5.4)
+ *
+ * Masks (page "SDPA란 무엇인가" section 1 bias B, section 4 trap 3 alignment;
+ * page "어텐션 메커니즘" sections 5 and 6).  With i' = i + (S - L) (bottom-right
+ * alignment, so a single decode query sees every cached key):
+ *   ATTN_MASK_NONE            every key visible
+ *   ATTN_MASK_CAUSAL          key j visible iff j <= i'
+ *   ATTN_MASK_SLIDING_WINDOW  key j visible iff 0 <= i' - j < window
+ * An additive float bias B[i, j] (0 or -inf; any finite value is added too)
+ * composes with every mask kind.  A row with no visible key and no sink yields
+ * out = 0 and lse = -inf (SDPA's fully-masked-row convention, page "SDPA란
+ * 무엇인가" section 4); with a sink it yields out = 0 and lse = s[hq].
+ *
+ * Grouped-query attention (page "SDPA란 무엇인가" section 5): query head hq reads
+ * KV head hq / (Hq / H).
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { ATTN_DOT = 0, ATTN_RBF = 1, ATTN_SINK = 2 } attn_mode;
+typedef enum {
+  ATTN_MASK_NONE = 0,
+  ATTN_MASK_CAUSAL = 1,
+  ATTN_MASK_SLIDING_WINDOW = 2
+} attn_mask_kind;
+typedef enum { ATTN_BF16 = 0, ATTN_FP32 = 1 } attn_dtype;
+
+/* Status codes.  Every entry point returns ATTN_OK (0) or one of these (< 0). */
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_NULL_POINTER = -1,   /* q, k, v or out is NULL, or sink is NULL with ATTN_SINK */
+  ATTN_ERR_BAD_SHAPE = -2,      /* N, Hq, H, L or S < 1, or a size overflows 64-bit indexing */
+  ATTN_ERR_GQA = -3,            /* Hq is not a multiple of H */
+  ATTN_ERR_HEAD_DIM = -4,       /* E or Ev not in {64, 128} */
+  ATTN_ERR_SCALE = -5,          /* scale not finite or <= 0 */
+  ATTN_ERR_MODE = -6,           /* mode out of range */
+  ATTN_ERR_MASK = -7,           /* mask_kind out of range */
+  ATTN_ERR_WINDOW = -8,         /* window < 1 with ATTN_MASK_SLIDING_WINDOW */
+  ATTN_ERR_SINK = -9,           /* ATTN_SINK given without sink logits */
+  ATTN_ERR_DTYPE = -10,         /* dtype out of range */
+  ATTN_ERR_ALIGNMENT = -11,     /* q, k, v, out or bias not 16-byte aligned; lse not 4-byte aligned */
+  ATTN_ERR_WORKSPACE = -12,     /* the library could not allocate its decode workspace */
+  ATTN_ERR_CUDA = -13,          /* a CUDA call or kernel launch failed */
+  ATTN_ERR_DEVICE_TIMEOUT = -14,/* a kernel gave up a bounded wait (see attn_device_status) */
+  ATTN_ERR_DEVICE = -15         /* the current device is not sm_100 */
+} attn_status;
+
+/*
+ * attn_fwd -- the fused attention forward.
+ *
+ * Arguments (all pointers are device memory owned by the caller; the library
+ * never frees or retains them beyond the call's stream work):
+ *   q     [N, Hq, L, E]  contiguous, dtype given by `dtype`
+ *   k     [N, H,  S, E]  contiguous
+ *   v     [N, H,  S, Ev] contiguous
+ *   out   [N, Hq, L, Ev] contiguous, written in the input dtype
+ *   lse   [N, Hq, L] float32, natural-log log-sum-exp of each row's logits,
+ *         the sink term included (NULL: not written)
+ *   scale        > 0; multiplies q.k (dot) or the squared distance (rbf)
+ *   mode         ATTN_DOT, ATTN_RBF, or ATTN_SINK (= ATTN_DOT with a required sink).
+ *                A non-NULL sink_logits applies the sink in any mode.
+ *   sink_logits  [Hq] float32 or NULL
+ *   mask_kind    attn_mask_kind; window = number of visible keys per query
+ *                (self included) for ATTN_MASK_SLIDING_WINDOW, ignored otherwise
+ *   bias         [L, S] float32 additive bias, broadcast over n and heads, or NULL
+ *   dtype        ATTN_BF16 (tensor-core path, fp32 accumulation) or ATTN_FP32
+ *                (exact fp32 FFMA path)
+ *   stream       a cudaStream_t (NULL = the legacy default stream)
+ *
+ * The call validates every argument first and launches nothing on error.  On
+ * success it enqueues its kernels on `stream` and returns without a host
+ * synchronisation.  bf16 calls with (Hq/H)*L <= 16 run the split-key decode
+ * path (partial kernel + combine kernel), which uses a library-owned device
+ * workspace allocated stream-ordered on first need and grown monotonically;
+ * all other bf16 calls run the single-kernel tcgen05 prefill path.
+ * Calls on different streams may run concurrently except decode calls, which
+ * share the workspace and must be ordered by the caller.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+             int N, int Hq, int H, int L, int S, int E, int Ev, float scale, int mode,
+             const float* sink_logits, int mask_kind, int window, const float* bias,
+             int dtype, void* stream);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+const char* attn_status_string(int status);
+
+/* Frees the decode workspace (synchronises the device first).  The next decode
+ * call allocates it again. */
+void attn_release_workspace(void);
+
+/*
+ * attn_device_status -- synchronises `stream`, then reads and clears the
+ * device-side status word.  Every wait inside the kernels (on a TMA transfer,
+ * a tensor-core commit or a sibling warp) is bounded; a wait that runs out
+ * makes its CTA record the fault here, drain its own in-flight copies and
+ * tensor-core work, release its tensor memory and exit.  Returns ATTN_OK,
+ * ATTN_ERR_DEVICE_TIMEOUT, or ATTN_ERR_CUDA if the synchronisation failed.
+ */
+int attn_device_status(void* stream);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,83 @@
+"""The C-ABI library on the host: it loads, exports every declared symbol, and
+rejects bad arguments before touching the GPU (no compute calls here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import attention_tiled_attn_b200 as attn
+from attention_tiled_attn_b200 import build as attn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_b200.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    attn_build.build()
+    return attn.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(attn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("attn_fwd", "attn_status_string", "attn_release_workspace", "attn_device_status", "attn_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    assert attn.status_string(0) == "ok"
+    for st in range(-15, 0):
+        s = attn.status_string(st)
+        assert s and s != "unknown status"
+    assert attn.status_string(-99) == "unknown status"
+    assert attn.version() == 10000
+
+
+P = 0x10000  # a 16-byte aligned fake device address; never dereferenced on the error paths
+
+
+def call(**kw):
+    a = dict(q=P, k=P, v=P, out=P, lse=P, N=1, Hq=2, H=1, L=8, S=8, E=64, Ev=64, scale=0.125, mode=0,
+             sink=None, mask_kind=0, window=0, bias=None, dtype=0, stream=None)
+    a.update(kw)
+    return attn.attn_fwd_raw(a["q"], a["k"], a["v"], a["out"], a["lse"], a["N"], a["Hq"], a["H"], a["L"], a["S"],
+                             a["E"], a["Ev"], a["scale"], a["mode"], a["sink"], a["mask_kind"], a["window"],
+                             a["bias"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), -1), (dict(v=None), -1), (dict(out=None), -1),
+    (dict(N=0), -2), (dict(L=0), -2), (dict(S=-3), -2), (dict(Hq=0), -2),
+    (dict(Hq=3, H=2), -3),
+    (dict(E=96), -4), (dict(Ev=32), -4), (dict(E=256), -4),
+    (dict(scale=0.0), -5), (dict(scale=-1.0), -5), (dict(scale=float("inf")), -5), (dict(scale=float("nan")), -5),
+    (dict(mode=3), -6), (dict(mode=-1), -6),
+    (dict(mask_kind=3), -7), (dict(mask_kind=2, window=0), -8),
+    (dict(mode=2, sink=None), -9),
+    (dict(dtype=2), -10),
+    (dict(q=P + 8), -11), (dict(out=P + 4), -11), (dict(bias=P + 8), -11), (dict(lse=P + 2), -11),
+    (dict(N=1 << 20, Hq=1 << 12, H=1 << 12), -2),
+    (dict(dtype=1, N=1, Hq=70000, H=70000), -2),
+])
+def test_argument_validation(lib, kw, status):
+    assert call(**kw) == status
+
+
+def test_python_binding_rejects_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn.attn_fwd(q, q, q, scale=0.1)

@@ -1,0 +1,151 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+the same seeded inputs.  Small cases compare every element; the reference
+workloads run at full size in the benchmark's launch configuration and are
+compared on sampled rows."""
+
+import numpy as np
+import pytest
+import torch
+
+import attention_tiled_attn_b200 as attn
+from synth import gpu as sgpu
+from synth import workloads as sw
+
+import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda_ready():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from attention_tiled_attn_b200 import build as b
+    b.build()
+    sgpu.build()
+    yield
+    assert attn.device_status() == 0, "a kernel recorded a bounded-wait timeout"
+
+
+R = gu.small_recipe
+
+PREFILL_CASES = [
+    R("p_dot_none_128", L=128, S=128),
+    R("p_dot_causal_300_e128_g2", L=300, S=300, E=128, Ev=128, Hq=4, H=2, mask_kind="causal"),
+    R("p_rbf_causal_257_sink", L=257, S=257, mode="rbf", mask_kind="causal", sink="fixed",
+      sink_values=(0.0, 1.0)),
+    R("p_dot_window100_515_g3_sink", L=515, S=515, Ev=128, Hq=6, H=2, mask_kind="window", window=100,
+      sink="normal"),
+    R("p_dot_causal_L200_S600_g4", L=200, S=600, E=128, Ev=64, Hq=8, H=2, mask_kind="causal"),
+    R("p_dot_causal_L300_S100_empty_rows", L=300, S=100, mask_kind="causal"),
+    R("p_dot_bias10_192", L=192, S=192, Hq=1, H=1, bias="random10"),
+    R("p_rbf_window64_400_g2_bias", L=400, S=400, Hq=4, H=2, mode="rbf", mask_kind="window", window=64,
+      bias="random10"),
+    R("p_rbf_registers_260", L=260, S=260, mode="rbf", mask_kind="causal", registers=4, key_lognormal=True,
+      sinusoid_pe=True, sink="normal"),
+    R("p_dot_L17_S1", L=17, S=1),
+    R("p_dot_causal_33_g16", L=33, S=33, Hq=16, H=1, mask_kind="causal"),
+    R("p_rbf_none_L128_S1000_e128", L=128, S=1000, E=128, Ev=128, mode="rbf", scale=0.05),
+    R("p_dot_window1_130", L=130, S=130, mask_kind="window", window=1),
+    R("p_dot_none_600_g2_e128_sink", L=600, S=600, E=128, Ev=128, Hq=4, H=2, N=2, sink="normal",
+      scale=0.0884),
+]
+
+FP32_CASES = [
+    R("f_dot_bias_130_e128", L=130, S=130, E=128, Ev=128, dtype="f32", bias="random10"),
+    R("f_rbf_window50_sink_g3", L=150, S=170, Hq=3, H=1, dtype="f32", mode="rbf", mask_kind="window", window=50,
+      sink="normal"),
+    R("f_dot_causal_70_g2_ev128", L=70, S=70, Ev=128, Hq=2, H=1, dtype="f32", mask_kind="causal"),
+    R("f_dot_causal_L1_S6", L=1, S=6, dtype="f32", mask_kind="causal"),
+    R("f_dot_causal_L40_S10_empty", L=40, S=10, dtype="f32", mask_kind="causal", sink="fixed",
+      sink_values=(0.5, -0.5)),
+]
+
+DECODE_CASES = [
+    R("d_L1_g4_S1000_sink", L=1, S=1000, E=128, Ev=128, N=2, Hq=12, H=3, sink="normal", scale=0.0884),
+    R("d_L1_g1_S5000_causal", L=1, S=5000, N=3, Hq=1, H=1, mask_kind="causal"),
+    R("d_L4_g4_S777_causal_sink", L=4, S=777, Hq=8, H=2, mask_kind="causal", sink="normal"),
+    R("d_L2_g2_S300_window_bias", L=2, S=300, Hq=2, H=1, mask_kind="window", window=50, bias="random10"),
+    R("d_L1_g8_S64", L=1, S=64, Hq=8, H=1),
+    R("d_L1_S1", L=1, S=1, Hq=2, H=2),
+    R("d_L3_g5_S129_e128_ev64", L=3, S=129, E=128, Ev=64, Hq=5, H=1),
+    R("d_many_units", L=1, S=200, N=40, Hq=16, H=8, sink="normal"),
+    R("d_L2_causal_S1_empty_row", L=2, S=1, Hq=2, H=2, mask_kind="causal"),
+]
+
+
+@pytest.mark.parametrize("r", PREFILL_CASES, ids=lambda r: r.name)
+def test_prefill_bf16_small(r):
+    gu.run_and_check_full(r)
+
+
+@pytest.mark.parametrize("r", FP32_CASES, ids=lambda r: r.name)
+def test_fp32_small(r):
+    gu.run_and_check_full(r)
+
+
+@pytest.mark.parametrize("r", DECODE_CASES, ids=lambda r: r.name)
+def test_decode_bf16_small(r):
+    assert (r.Hq // r.H) * r.L <= 16
+    gu.run_and_check_full(r)
+
+
+def test_tiny_reference_workload_fp32():
+    gu.run_and_check_full(sw.RECIPES["tiny_rbf_sink_causal_f32"])
+
+
+def test_output_canaries():
+    """Nothing is written past the end of out and lse."""
+    r = R("canary", L=300, S=300, E=128, Ev=128, Hq=4, H=2, mask_kind="causal", sink="normal")
+    host = sw.generate(r)
+    q, k, v = (sgpu.to_device(host[x], r) for x in ("q", "k", "v"))
+    sink = torch.from_numpy(host["sink"]).cuda()
+    for shape_l in (r.L, 1):
+        qq = q[:, :, :shape_l].contiguous()
+        n_out = r.N * r.Hq * shape_l * r.Ev
+        n_lse = r.N * r.Hq * shape_l
+        obuf = torch.full((n_out + 4096,), 7.0, dtype=torch.bfloat16, device="cuda")
+        lbuf = torch.full((n_lse + 4096,), 7.0, dtype=torch.float32, device="cuda")
+        out = obuf[:n_out].view(r.N, r.Hq, shape_l, r.Ev)
+        lse = lbuf[:n_lse].view(r.N, r.Hq, shape_l)
+        attn.attn_fwd(qq, k, v, scale=r.scale, sink=sink, mask_kind="causal", out=out, lse=lse)
+        torch.cuda.synchronize()
+        assert torch.all(obuf[n_out:] == 7.0) and torch.all(lbuf[n_lse:] == 7.0)
+
+
+def test_repeat_calls_are_deterministic():
+    r = R("det", L=256, S=256, Hq=4, H=2, mask_kind="causal", sink="normal")
+    host = sw.generate(r)
+    t = {x: sgpu.to_device(host[x], r) for x in ("q", "k", "v")}
+    t["sink"], t["bias"] = torch.from_numpy(host["sink"]).cuda(), None
+    a, la = gu.run_gpu(r, t)
+    b, lb = gu.run_gpu(r, t)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+# ---------------------------------------------------------------------------
+# the reference workloads at full size, sampled rows
+# ---------------------------------------------------------------------------
+
+FULL = ["dot_causal_2k_bf16", "dot_bias10_2k_f32", "rbf_registers_4k_bf16", "sink_gqa_window_16k_bf16",
+        "decode_sink_gqa_128k_bf16"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_reference_workload_full_size(name):
+    r = sw.RECIPES[name]
+    t = sgpu.generate_on_device(r)
+    out, lse = gu.run_gpu(r, t)
+    assert torch.isfinite(out.float()).all()
+    rng = np.random.default_rng(sum(map(ord, name)))
+    units = [(0, 0), (r.N - 1, r.Hq - 1), (int(rng.integers(r.N)), int(rng.integers(r.Hq)))]
+    if name.startswith("decode"):
+        units = units[:2]
+    for n, hq in units:
+        rows = gu.sample_rows(r.L, rng, count=12 if r.L > 1 else 0)
+        ref_out, ref_lse = gu.oracle_rows(r, n, hq, rows)
+        got = gu.out_to_f64(out[n, hq, rows])
+        got_lse = lse[n, hq, rows].cpu().numpy()
+        gu.compare(r, got, got_lse, ref_out, ref_lse, f"{name} n={n} hq={hq}")
+    del t, out, lse
+    torch.cuda.empty_cache()

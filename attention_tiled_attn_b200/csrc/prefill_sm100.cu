@@ -9,6 +9,7 @@
 //   warp  8     TMA producer: Q tiles once, then K and V tiles through rings
 //   warp  9     tcgen05 issuer: S_t = Q_t K^T into TMEM, O_t += P_t V from TMEM
 //   warp 10     key-norm warp (RBF only): ||k_j||^2 of each key tile from smem
+//   warp 11     idle (completes the third warpgroup of the register split)
 //
 // Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 and O_1 after
 // them.  P_t (bf16, two per column) overwrites the first 64 columns of S_t.
@@ -71,22 +72,31 @@ struct Cfg {
   static constexpr int OFF_KN = OFF_V + NV * V_BYTES;
   static constexpr int OFF_BAR = OFF_KN + (RBF ? NKN * BN * 4 : 0);
   // barrier indices
-  static constexpr int B_Q = 0;
-  static constexpr int B_KFULL = 1;
+  static constexpr int B_QFULL = 0;
+  static constexpr int B_QEMPTY = 1;
+  static constexpr int B_KFULL = 2;
   static constexpr int B_KEMPTY = B_KFULL + NK;
   static constexpr int B_VFULL = B_KEMPTY + NK;
   static constexpr int B_VEMPTY = B_VFULL + NV;
   static constexpr int B_SFULL = B_VEMPTY + NV;
   static constexpr int B_PFULL = B_SFULL + 2;
   static constexpr int B_OFULL = B_PFULL + 2;
-  static constexpr int B_KNFULL = B_OFULL + 2;
+  static constexpr int B_OEMPTY = B_OFULL + 2;
+  static constexpr int B_KNFULL = B_OEMPTY + 2;
   static constexpr int B_KNEMPTY = B_KNFULL + NKN;
   static constexpr int B_DRAIN = B_KNEMPTY + NKN;
   static constexpr int NUM_BARS = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + base alignment slack
-  static constexpr int NUM_WARPS = RBF ? 11 : 10;
+  static constexpr int NUM_WARPS = 12;  // three warpgroups
   static constexpr int THREADS = NUM_WARPS * 32;
+  // Register split after launch (setmaxnreg): the softmax warpgroups grow to
+  // REG_SOFTMAX, the producer / issuer / key-norm warpgroup shrinks to
+  // REG_OTHER.  256 * 216 + 128 * 72 = 168 * 384, the launch budget; the host
+  // refuses to launch if the compiled count is lower (the .inc would never
+  // be satisfied).
+  static constexpr uint32_t REG_SOFTMAX = 216;
+  static constexpr uint32_t REG_OTHER = 72;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, EV, 1);
@@ -129,6 +139,57 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+// One work item: two query tiles sharing a K/V stream, and the union of their key-tile ranges.
+struct Item {
+  int n, kvh;
+  TileInfo tile[2];
+  int u_lo, u_hi;
+};
+
+__device__ __forceinline__ void decode_item(const PrefillParams& p, int item, Item& w) {
+  if (p.head_pairs) {
+    const int hp_per = p.group / 2;
+    const int per_rb = p.N * p.H * hp_per;
+    const int rb = p.n_rb - 1 - item / per_rb;  // heavy (late) row blocks first
+    const int r = item % per_rb;
+    w.n = r / (p.H * hp_per);
+    const int rem = r % (p.H * hp_per);
+    w.kvh = rem / hp_per;
+    const int hq0 = w.kvh * p.group + 2 * (rem % hp_per);
+    w.tile[0] = {1, hq0, rb * BM, 0, 0};
+    w.tile[1] = {1, hq0 + 1, rb * BM, 0, 0};
+  } else {
+    const int n_rp = (p.n_rb + 1) / 2;
+    const int per_rp = p.N * p.Hq;
+    const int rp = n_rp - 1 - item / per_rp;
+    const int r = item % per_rp;
+    w.n = r / p.Hq;
+    const int hq = r % p.Hq;
+    w.kvh = hq / p.group;
+    w.tile[0] = {1, hq, 2 * rp * BM, 0, 0};
+    w.tile[1] = {(2 * rp + 1) * BM < p.L ? 1 : 0, hq, (2 * rp + 1) * BM, 0, 0};
+  }
+  tile_range(p, w.tile[0]);
+  tile_range(p, w.tile[1]);
+  const bool h0 = w.tile[0].jb_hi > w.tile[0].jb_lo;
+  const bool h1 = w.tile[1].jb_hi > w.tile[1].jb_lo;
+  w.u_lo = w.u_hi = 0;
+  if (h0 && h1) {
+    w.u_lo = min(w.tile[0].jb_lo, w.tile[1].jb_lo);
+    w.u_hi = max(w.tile[0].jb_hi, w.tile[1].jb_hi);
+  } else if (h0) {
+    w.u_lo = w.tile[0].jb_lo;
+    w.u_hi = w.tile[0].jb_hi;
+  } else if (h1) {
+    w.u_lo = w.tile[1].jb_lo;
+    w.u_hi = w.tile[1].jb_hi;
+  }
+}
+
+// Items are numbered heaviest first; CTA b takes, in round k, item k*G + b
+// (k even) or k*G + G-1-b (k odd), so the heavy items spread evenly.
+__device__ __forceinline__ int snake_item(int b, int k, int G) { return k * G + ((k & 1) ? (G - 1 - b) : b); }
+
 template <int E, int EV, bool RBF>
 __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -144,55 +205,14 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- work item --------------------------------------------------------
-  int n, kvh;
-  TileInfo tile[2];
-  {
-    const int item = blockIdx.x;
-    if (p.head_pairs) {
-      const int hp_per = p.group / 2;
-      const int per_rb = p.N * p.H * hp_per;
-      const int rb = p.n_rb - 1 - item / per_rb;  // heavy (late) row blocks first
-      const int r = item % per_rb;
-      n = r / (p.H * hp_per);
-      const int rem = r % (p.H * hp_per);
-      kvh = rem / hp_per;
-      const int hq0 = kvh * p.group + 2 * (rem % hp_per);
-      tile[0] = {1, hq0, rb * BM, 0, 0};
-      tile[1] = {1, hq0 + 1, rb * BM, 0, 0};
-    } else {
-      const int n_rp = (p.n_rb + 1) / 2;
-      const int per_rp = p.N * p.Hq;
-      const int rp = n_rp - 1 - item / per_rp;
-      const int r = item % per_rp;
-      n = r / p.Hq;
-      const int hq = r % p.Hq;
-      kvh = hq / p.group;
-      tile[0] = {1, hq, 2 * rp * BM, 0, 0};
-      tile[1] = {(2 * rp + 1) * BM < p.L ? 1 : 0, hq, (2 * rp + 1) * BM, 0, 0};
-    }
-    tile_range(p, tile[0]);
-    tile_range(p, tile[1]);
-  }
-  const bool has0 = tile[0].jb_hi > tile[0].jb_lo;
-  const bool has1 = tile[1].jb_hi > tile[1].jb_lo;
-  int u_lo = 0, u_hi = 0;
-  if (has0 && has1) {
-    u_lo = min(tile[0].jb_lo, tile[1].jb_lo);
-    u_hi = max(tile[0].jb_hi, tile[1].jb_hi);
-  } else if (has0) {
-    u_lo = tile[0].jb_lo;
-    u_hi = tile[0].jb_hi;
-  } else if (has1) {
-    u_lo = tile[1].jb_lo;
-    u_hi = tile[1].jb_hi;
-  }
+  const int G = gridDim.x;
+  const int b = blockIdx.x;
 
   // ---- setup ------------------------------------------------------------
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(bar(C::B_Q), 1);
+    mbar_init(bar(C::B_QFULL), 1);
+    mbar_init(bar(C::B_QEMPTY), 1);
     for (int s = 0; s < C::NK; ++s) {
       mbar_init(bar(C::B_KFULL + s), 1);
       mbar_init(bar(C::B_KEMPTY + s), RBF ? 2 : 1);
@@ -205,6 +225,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
       mbar_init(bar(C::B_SFULL + t), 1);
       mbar_init(bar(C::B_PFULL + t), 128);
       mbar_init(bar(C::B_OFULL + t), 1);
+      mbar_init(bar(C::B_OEMPTY + t), 128);
     }
     for (int s = 0; s < C::NKN; ++s) {
       mbar_init(bar(C::B_KNFULL + s), 32);
@@ -222,106 +243,125 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 8) reg_dealloc<C::REG_OTHER>();
   if (warp == 8) {
     // ================= TMA producer =================
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      uint32_t qbytes = (has0 ? C::Q_BYTES : 0) + (has1 ? C::Q_BYTES : 0);
-      if (qbytes) {
-        mbar_arrive_expect_tx(bar(C::B_Q), qbytes);
-        for (int t = 0; t < 2; ++t) {
-          if (!(t == 0 ? has0 : has1)) continue;
-          for (int b = 0; b < E / 64; ++b)
-            tma_load_3d(sb + C::OFF_Q + t * C::Q_BYTES + b * (BM * 128), &tm_q, bar(C::B_Q), b * 64,
-                        tile[t].r0, n * p.Hq + tile[t].hq);
+      uint32_t gk = 0;   // key tiles loaded so far by this CTA (K and V rings advance together)
+      uint32_t qc = 0;   // items whose Q was loaded
+      bool ok = true;
+      for (int k = 0; ok && k * G < p.n_items; ++k) {
+        const int item = snake_item(b, k, G);
+        if (item >= p.n_items) continue;
+        Item w;
+        decode_item(p, item, w);
+        if (w.u_hi <= w.u_lo) continue;
+        const bool h0 = w.tile[0].jb_hi > w.tile[0].jb_lo, h1 = w.tile[1].jb_hi > w.tile[1].jb_lo;
+        bool q_pending = true;
+        for (int jb = w.u_lo; jb < w.u_hi; ++jb, ++gk) {
+          const uint32_t ks = gk % C::NK, vs = gk % C::NV;
+          if (!wait_bar(bar(C::B_KEMPTY + ks), ((gk / C::NK) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::B_KFULL + ks), C::K_BYTES);
+          for (int bb = 0; bb < E / 64; ++bb)
+            tma_load_3d(sb + C::OFF_K + ks * C::K_BYTES + bb * (BN * 128), &tm_k, bar(C::B_KFULL + ks), bb * 64,
+                        jb * BN, w.n * p.H + w.kvh);
+          if (q_pending) {
+            // the item's first K tile is in flight; now wait for the previous item's last QK^T
+            q_pending = false;
+            if (!wait_bar(bar(C::B_QEMPTY), (qc & 1) ^ 1, abort_flag)) {
+              ok = false;
+              ++gk;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(C::B_QFULL), (h0 ? C::Q_BYTES : 0) + (h1 ? C::Q_BYTES : 0));
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (!(t == 0 ? h0 : h1)) continue;
+              for (int bb = 0; bb < E / 64; ++bb)
+                tma_load_3d(sb + C::OFF_Q + t * C::Q_BYTES + bb * (BM * 128), &tm_q, bar(C::B_QFULL), bb * 64,
+                            w.tile[t].r0, w.n * p.Hq + w.tile[t].hq);
+            }
+            ++qc;
+          }
+          if (!wait_bar(bar(C::B_VEMPTY + vs), ((gk / C::NV) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            ++gk;  // this K load is in flight and must be drained
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::B_VFULL + vs), C::V_BYTES);
+          for (int bb = 0; bb < EV / 64; ++bb)
+            tma_load_3d(sb + C::OFF_V + vs * C::V_BYTES + bb * (BN * 128), &tm_v, bar(C::B_VFULL + vs), bb * 64,
+                        jb * BN, w.n * p.H + w.kvh);
         }
       }
-      int last_k_phase[C::NK], last_v_phase[C::NV];
-      for (int s = 0; s < C::NK; ++s) last_k_phase[s] = -1;
-      for (int s = 0; s < C::NV; ++s) last_v_phase[s] = -1;
-      for (int jb = u_lo; jb < u_hi; ++jb) {
-        const int idx = jb - u_lo;
-        const int ks = idx % C::NK;
-        const uint32_t kph = (idx / C::NK) & 1;
-        if (!wait_bar(bar(C::B_KEMPTY + ks), kph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::B_KFULL + ks), C::K_BYTES);
-        for (int b = 0; b < E / 64; ++b)
-          tma_load_3d(sb + C::OFF_K + ks * C::K_BYTES + b * (BN * 128), &tm_k, bar(C::B_KFULL + ks), b * 64,
-                      jb * BN, n * p.H + kvh);
-        last_k_phase[ks] = kph;
-        const int vs = idx % C::NV;
-        const uint32_t vph = (idx / C::NV) & 1;
-        if (!wait_bar(bar(C::B_VEMPTY + vs), vph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::B_VFULL + vs), C::V_BYTES);
-        for (int b = 0; b < EV / 64; ++b)
-          tma_load_3d(sb + C::OFF_V + vs * C::V_BYTES + b * (BN * 128), &tm_v, bar(C::B_VFULL + vs), b * 64,
-                      jb * BN, n * p.H + kvh);
-        last_v_phase[vs] = vph;
-      }
-      // drain: every issued copy has landed before the CTA may exit
-      if (qbytes) mbar_wait(bar(C::B_Q), 0);
-      for (int s = 0; s < C::NK; ++s)
-        if (last_k_phase[s] >= 0) mbar_wait(bar(C::B_KFULL + s), last_k_phase[s]);
-      for (int s = 0; s < C::NV; ++s)
-        if (last_v_phase[s] >= 0) mbar_wait(bar(C::B_VFULL + s), last_v_phase[s]);
+      // drain: the most recent phase of every ring slot (and Q) has landed before exit
+      if (qc) mbar_wait(bar(C::B_QFULL), (qc - 1) & 1);
+      for (uint32_t j = (gk > C::NK ? gk - C::NK : 0); j < gk; ++j) mbar_wait(bar(C::B_KFULL + j % C::NK), (j / C::NK) & 1);
+      for (uint32_t j = (gk > C::NV ? gk - C::NV : 0); j < gk; ++j) mbar_wait(bar(C::B_VFULL + j % C::NV), (j / C::NV) & 1);
     }
   } else if (warp == 9) {
     // ================= tcgen05 issuer =================
     if (lane == 0) {
+      uint32_t gk = 0, qc = 0;
+      uint32_t pv_count0 = 0, pv_count1 = 0;  // PVs issued per tile (p_full phases)
+      uint32_t oc0 = 0, oc1 = 0;              // items with an O accumulation per tile
       bool ok = true;
-      if (u_hi > u_lo) ok = wait_bar(bar(C::B_Q), 0, abort_flag);
-      tc_fence_after();
-      int pend[2] = {-1, -1};
-      int pv_count[2] = {0, 0};
-      int v_waited = u_lo - 1;  // highest key tile whose V landing was awaited
-      int v_cur = -1, v_cur_uses = 0;
-
-      auto issue_pv = [&](int t, int jbp) -> bool {
-        const int idxp = jbp - u_lo;
-        const int vs = idxp % C::NV;
-        if (jbp > v_waited) {
-          if (!wait_bar(bar(C::B_VFULL + vs), (idxp / C::NV) & 1, abort_flag)) return false;
-          v_waited = jbp;
-        }
-        if (!wait_bar(bar(C::B_PFULL + t), pv_count[t] & 1, abort_flag)) return false;
+      for (int k = 0; ok && k * G < p.n_items; ++k) {
+        const int item = snake_item(b, k, G);
+        if (item >= p.n_items) continue;
+        Item w;
+        decode_item(p, item, w);
+        if (w.u_hi <= w.u_lo) continue;
+        if (!wait_bar(bar(C::B_QFULL), qc & 1, abort_flag)) break;
+        ++qc;
         tc_fence_after();
-        const uint32_t d = tmem + 256 + t * EV;
-        const uint32_t a = tmem + t * 128;
-        const uint32_t vbase = sb + C::OFF_V + vs * C::V_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // B = V tile, MN-major: 16 keys per step = 16 rows of 128 B; second 64-column box at +BN*128
-          const uint64_t bdesc = smem_desc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
-          mma_ts(d, a + kk * 8, bdesc, C::IDESC_PV, (pv_count[t] > 0 || kk > 0) ? 1u : 0u);
-        }
-        pv_count[t]++;
-        const int uses = (in_range(tile[0], jbp) ? 1 : 0) + (in_range(tile[1], jbp) ? 1 : 0);
-        if (jbp != v_cur) {
-          v_cur = jbp;
-          v_cur_uses = 0;
-        }
-        if (++v_cur_uses == uses) mma_commit(bar(C::B_VEMPTY + vs));
-        return true;
-      };
+        const uint32_t gbase = gk;
+        int pend0 = -1, pend1 = -1;
+        bool first0 = true, first1 = true;
+        int v_waited = w.u_lo - 1, v_cur = -1, v_cur_uses = 0;
 
-      for (int jb = u_lo; ok && jb < u_hi; ++jb) {
-        const int idx = jb - u_lo;
-        const int ks = idx % C::NK;
-        if (!wait_bar(bar(C::B_KFULL + ks), (idx / C::NK) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!in_range(tile[t], jb)) continue;
-          if (pend[t] >= 0) {
-            if (!issue_pv(t, pend[t])) {
-              ok = false;
-              break;
-            }
+        auto issue_pv = [&](int t, int jbp) -> bool {
+          const uint32_t gp = gbase + (jbp - w.u_lo);
+          const uint32_t vs = gp % C::NV;
+          if (jbp > v_waited) {
+            if (!wait_bar(bar(C::B_VFULL + vs), (gp / C::NV) & 1, abort_flag)) return false;
+            v_waited = jbp;
           }
+          uint32_t& pvc = t ? pv_count1 : pv_count0;
+          bool& first = t ? first1 : first0;
+          const uint32_t oc = t ? oc1 : oc0;
+          if (!wait_bar(bar(C::B_PFULL + t), pvc & 1, abort_flag)) return false;
+          if (first && oc > 0) {
+            // the previous item's epilogue must have read O_t before it is overwritten
+            if (!wait_bar(bar(C::B_OEMPTY + t), (oc - 1) & 1, abort_flag)) return false;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + 256 + t * EV;
+          const uint32_t a = tmem + t * 128;
+          const uint32_t vbase = sb + C::OFF_V + vs * C::V_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // B = V tile, MN-major: 16 keys per step = 16 rows of 128 B; second 64-column box at +BN*128
+            const uint64_t bdesc = smem_desc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
+            mma_ts(d, a + kk * 8, bdesc, C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+          }
+          first = false;
+          ++pvc;
+          const int uses = (in_range(w.tile[0], jbp) ? 1 : 0) + (in_range(w.tile[1], jbp) ? 1 : 0);
+          if (jbp != v_cur) {
+            v_cur = jbp;
+            v_cur_uses = 0;
+          }
+          if (++v_cur_uses == uses) mma_commit(bar(C::B_VEMPTY + vs));
+          return true;
+        };
+        auto issue_qk = [&](int t, uint32_t ks) {
           const uint32_t d = tmem + t * 128;
           const uint32_t qbase = sb + C::OFF_Q + t * C::Q_BYTES;
           const uint32_t kbase = sb + C::OFF_K + ks * C::K_BYTES;
@@ -333,24 +373,46 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
             mma_ss(d, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar(C::B_SFULL + t));
-          pend[t] = jb;
+        };
+
+        for (int jb = w.u_lo; ok && jb < w.u_hi; ++jb, ++gk) {
+          const uint32_t ks = gk % C::NK;
+          if (!wait_bar(bar(C::B_KFULL + ks), (gk / C::NK) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (in_range(w.tile[0], jb)) {
+            if (pend0 >= 0 && !issue_pv(0, pend0)) { ok = false; break; }
+            issue_qk(0, ks);
+            pend0 = jb;
+          }
+          if (in_range(w.tile[1], jb)) {
+            if (pend1 >= 0 && !issue_pv(1, pend1)) { ok = false; break; }
+            issue_qk(1, ks);
+            pend1 = jb;
+          }
+          mma_commit(bar(C::B_KEMPTY + ks));
+          if (!in_range(w.tile[0], jb) && !in_range(w.tile[1], jb)) {
+            // a key tile neither query tile reads: let its V copy land, then free the slot
+            const uint32_t vs = gk % C::NV;
+            if (!wait_bar(bar(C::B_VFULL + vs), (gk / C::NV) & 1, abort_flag)) { ok = false; break; }
+            mma_commit(bar(C::B_VEMPTY + vs));
+            if (jb > v_waited) v_waited = jb;
+          }
         }
-        if (ok) mma_commit(bar(C::B_KEMPTY + ks));
-        if (ok && !in_range(tile[0], jb) && !in_range(tile[1], jb)) {
-          // a key tile neither query tile reads: let its V copy land, then free the slot
-          const int vs = idx % C::NV;
-          if (!wait_bar(bar(C::B_VFULL + vs), (idx / C::NV) & 1, abort_flag)) ok = false;
-          else mma_commit(bar(C::B_VEMPTY + vs));
-          if (jb > v_waited) v_waited = jb;
+        if (!ok) break;
+        mma_commit(bar(C::B_QEMPTY));  // all QK^T of this item issued: Q may be replaced
+        if (pend0 >= 0) {
+          if (!issue_pv(0, pend0)) break;
+          mma_commit(bar(C::B_OFULL + 0));
+          ++oc0;
         }
-      }
-      for (int t = 0; t < 2 && ok; ++t) {
-        if (pend[t] < 0) continue;
-        if (!issue_pv(t, pend[t])) {
-          ok = false;
-          break;
+        if (pend1 >= 0) {
+          if (!issue_pv(1, pend1)) break;
+          mma_commit(bar(C::B_OFULL + 1));
+          ++oc1;
         }
-        mma_commit(bar(C::B_OFULL + t));
       }
       // drain: all issued tensor-core work completes before TMEM is released
       mma_commit(bar(C::B_DRAIN));
@@ -358,223 +420,261 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
     }
   } else if (RBF && warp == 10) {
     // ================= key-norm warp (RBF) =================
-    for (int jb = u_lo; jb < u_hi; ++jb) {
-      const int idx = jb - u_lo;
-      const int ks = idx % C::NK;
-      const int slot = idx % C::NKN;
-      if (!wait_bar(bar(C::B_KFULL + ks), (idx / C::NK) & 1, abort_flag)) break;
-      if (!wait_bar(bar(C::B_KNEMPTY + slot), ((idx / C::NKN) & 1) ^ 1, abort_flag)) break;
-      const uint8_t* ktile = sp + C::OFF_K + ks * C::K_BYTES;
-      float* kn = reinterpret_cast<float*>(sp + C::OFF_KN) + slot * BN;
+    uint32_t gk = 0;
+    bool ok = true;
+    for (int k = 0; ok && k * G < p.n_items; ++k) {
+      const int item = snake_item(b, k, G);
+      if (item >= p.n_items) continue;
+      Item w;
+      decode_item(p, item, w);
+      for (int jb = w.u_lo; jb < w.u_hi; ++jb, ++gk) {
+        const uint32_t ks = gk % C::NK;
+        const uint32_t slot = gk % C::NKN;
+        const bool w1 = wait_bar(bar(C::B_KFULL + ks), (gk / C::NK) & 1, abort_flag);
+        const bool w2 = w1 && wait_bar(bar(C::B_KNEMPTY + slot), ((gk / C::NKN) & 1) ^ 1, abort_flag);
+        if (!__all_sync(0xffffffffu, w2)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* ktile = sp + C::OFF_K + ks * C::K_BYTES;
+        float* kn = reinterpret_cast<float*>(sp + C::OFF_KN) + slot * BN;
 #pragma unroll
-      for (int rr = 0; rr < BN / 32; ++rr) {
-        const int r = lane + 32 * rr;
-        float acc = 0.f;
+        for (int rr = 0; rr < BN / 32; ++rr) {
+          const int r = lane + 32 * rr;
+          float acc = 0.f;
 #pragma unroll
-        for (int b = 0; b < E / 64; ++b) {
+          for (int bb = 0; bb < E / 64; ++bb) {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 w = *reinterpret_cast<const uint4*>(ktile + b * (BN * 128) + r * 128 + ((c ^ (r & 7)) << 4));
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+            for (int c = 0; c < 8; ++c) {
+              const uint4 wv =
+                  *reinterpret_cast<const uint4*>(ktile + bb * (BN * 128) + r * 128 + ((c ^ (r & 7)) << 4));
+              const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float lo = __uint_as_float(ws[e] << 16);
-              const float hi = __uint_as_float(ws[e] & 0xFFFF0000u);
-              acc = fmaf(lo, lo, acc);
-              acc = fmaf(hi, hi, acc);
+              for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(ws[e] << 16);
+                const float hi = __uint_as_float(ws[e] & 0xFFFF0000u);
+                acc = fmaf(lo, lo, acc);
+                acc = fmaf(hi, hi, acc);
+              }
             }
           }
+          kn[r] = acc * p.c_kn;
         }
-        kn[r] = acc * p.c_kn;
+        __syncwarp();
+        mbar_arrive(bar(C::B_KNFULL + slot));
+        if (lane == 0) mbar_arrive(bar(C::B_KEMPTY + ks));
       }
-      __syncwarp();
-      mbar_arrive(bar(C::B_KNFULL + slot));
-      if (lane == 0) mbar_arrive(bar(C::B_KEMPTY + ks));
     }
   } else if (warp < 8) {
     // ================= softmax warpgroups =================
+    reg_alloc<C::REG_SOFTMAX>();
     const int t = warp >> 2;
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
-    const TileInfo T = t ? tile[1] : tile[0];
-    const int i = T.r0 + row;
-    const int off = p.S - p.L;
-    const int lo_i = (p.mask_kind == MASK_WINDOW) ? (i + off - p.window + 1) : 0;
-    const int hi_i = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, i + off + 1);
-    const int first_row_hi = T.r0 + off + 1;               // key limit of the tile's first row
-    const int last_row_lo = min(T.r0 + BM - 1, p.L - 1) + off - p.window + 1;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t t_s = tmem + lane_base + t * 128;
     const uint32_t t_o = tmem + lane_base + 256 + t * EV;
     const bool has_bias = p.bias != nullptr;
-    const float* bias_row = has_bias && i < p.L ? p.bias + static_cast<size_t>(i) * p.S : nullptr;
-
-    float m_run = -INFINITY, l_run = 0.f;
-    int it = 0;
+    const int off = p.S - p.L;
+    uint32_t gk = 0;   // union key tiles seen (key-norm ring)
+    uint32_t sc = 0;   // S tiles consumed (s_full / p_full phases)
+    uint32_t oc = 0;   // O accumulations consumed (o_full phases)
     bool ok = true;
-    for (int jb = u_lo; jb < u_hi; ++jb) {
-      const int idx = jb - u_lo;
-      const int slot = idx % C::NKN;
-      if (RBF) {
-        const bool w = wait_bar(bar(C::B_KNFULL + slot), (idx / C::NKN) & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) {
-          ok = false;
-          break;
-        }
-      }
-      if (!in_range(T, jb)) {
-        if (RBF) mbar_arrive(bar(C::B_KNEMPTY + slot));
-        continue;
-      }
-      {
-        const bool w = wait_bar(bar(C::B_SFULL + t), it & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) {
-          ok = false;
-          break;
-        }
-      }
-      tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-      tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-      tmem_wait_ld();
-      float* z = reinterpret_cast<float*>(sr);
+    for (int k = 0; ok && k * G < p.n_items; ++k) {
+      const int item = snake_item(b, k, G);
+      if (item >= p.n_items) continue;
+      Item w;
+      decode_item(p, item, w);
+      const TileInfo T = t ? w.tile[1] : w.tile[0];
+      const int i = T.r0 + row;
+      const int lo_i = (p.mask_kind == MASK_WINDOW) ? (i + off - p.window + 1) : 0;
+      const int hi_i = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, i + off + 1);
+      const int first_row_hi = T.r0 + off + 1;  // key limit of the tile's first row
+      const int last_row_lo = min(T.r0 + BM - 1, p.L - 1) + off - p.window + 1;
+      const float* bias_row = has_bias && i < p.L ? p.bias + static_cast<size_t>(i) * p.S : nullptr;
 
-      const int k0 = jb * BN;
-      const bool need_mask = ((k0 + BN) > p.S) ||
-                             (p.mask_kind != MASK_NONE && (k0 + BN) > first_row_hi) ||
-                             (p.mask_kind == MASK_WINDOW && k0 < last_row_lo);
-      const bool scaled = RBF || need_mask || has_bias;
-      if (RBF) {
-        const float* kn = reinterpret_cast<const float*>(sp + C::OFF_KN) + slot * BN;
-#pragma unroll
-        for (int c = 0; c < BN; c += 4) {
-          const float4 kv = *reinterpret_cast<const float4*>(kn + c);
-          z[c + 0] = fmaf(z[c + 0], p.c_rbf, -kv.x);
-          z[c + 1] = fmaf(z[c + 1], p.c_rbf, -kv.y);
-          z[c + 2] = fmaf(z[c + 2], p.c_rbf, -kv.z);
-          z[c + 3] = fmaf(z[c + 3], p.c_rbf, -kv.w);
-        }
-        __syncwarp();
-        mbar_arrive(bar(C::B_KNEMPTY + slot));
-      } else if (scaled) {
-#pragma unroll
-        for (int c = 0; c < BN; ++c) z[c] *= p.c_dot;
-      }
-      if (need_mask) {
-#pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const int key = k0 + c;
-          if (key < lo_i || key >= hi_i) z[c] = -INFINITY;
-        }
-      }
-      if (has_bias && bias_row != nullptr) {
-#pragma unroll 8
-        for (int c = 0; c < BN; ++c) {
-          const int key = k0 + c;
-          if (key < p.S) z[c] = fmaf(__ldg(bias_row + key), LOG2E, z[c]);
-        }
-      }
-      float mt = z[0];
-#pragma unroll
-      for (int c = 1; c < BN; ++c) mt = fmaxf(mt, z[c]);
-      if (!scaled) mt *= p.c_dot;
-
-      const float m_new = fmaxf(m_run, mt);
-      const bool rescale = m_new > m_run + RESCALE_THRESHOLD;
-      if (__any_sync(0xffffffffu, rescale)) {
-        const float alpha = rescale ? ex2(m_run - m_new) : 1.f;
-        if (rescale) {
-          l_run *= alpha;
-          m_run = m_new;
-        }
-        if (it > 0) {
-#pragma unroll 1
-          for (int c = 0; c < EV; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(t_o + c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(t_o + c, o);
+      float m_run = -INFINITY, l_run = 0.f;
+      int it = 0;
+      for (int jb = w.u_lo; jb < w.u_hi; ++jb, ++gk) {
+        const uint32_t slot = gk % C::NKN;
+        if (RBF) {
+          const bool wk = wait_bar(bar(C::B_KNFULL + slot), (gk / C::NKN) & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, wk)) {
+            ok = false;
+            break;
           }
         }
-      }
-      const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-      float rs = 0.f;
-      uint32_t pk[64];
-      if (scaled) {
-#pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          const float p0 = ex2(z[c] - mu);
-          const float p1 = ex2(z[c + 1] - mu);
-          rs += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
+        if (!in_range(T, jb)) {
+          if (RBF) mbar_arrive(bar(C::B_KNEMPTY + slot));
+          continue;
         }
-      } else {
-        const float nm = -mu;
-#pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          const float p0 = ex2(fmaf(z[c], p.c_dot, nm));
-          const float p1 = ex2(fmaf(z[c + 1], p.c_dot, nm));
-          rs += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
+        {
+          const bool ws = wait_bar(bar(C::B_SFULL + t), sc & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, ws)) {
+            ok = false;
+            break;
+          }
         }
-      }
-      l_run += rs;
-      tmem_st32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_PFULL + t));
-      ++it;
-    }
-
-    // ---- epilogue ----
-    ok = __all_sync(0xffffffffu, ok);
-    if (T.active && ok) {
-      bool have_o = it > 0;
-      if (have_o) {
-        have_o = __all_sync(0xffffffffu, wait_bar(bar(C::B_OFULL + t), 0, abort_flag));
+        ++sc;
         tc_fence_after();
-      }
-      const float s2 = p.sink ? p.sink[T.hq] * LOG2E : -INFINITY;
-      const float M2 = fmaxf(m_run, s2);
-      float inv = 0.f, lse2 = -INFINITY;
-      if (M2 != -INFINITY) {
-        const float a = ex2(m_run - M2);
-        const float lp = l_run * a + ex2(s2 - M2);
-        if (lp > 0.f) {
-          inv = a / lp;
-          lse2 = M2 + __log2f(lp);
+        // S row -> registers (no array address is ever taken, so all of it stays in registers)
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(t_s + 0, r0);
+        tmem_ld32(t_s + 32, r1);
+        tmem_ld32(t_s + 64, r2);
+        tmem_ld32(t_s + 96, r3);
+        tmem_wait_ld();
+        float z[BN];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          z[e] = __uint_as_float(r0[e]);
+          z[32 + e] = __uint_as_float(r1[e]);
+          z[64 + e] = __uint_as_float(r2[e]);
+          z[96 + e] = __uint_as_float(r3[e]);
         }
-      }
-      const bool row_ok = i < p.L;
-      const size_t orow = (static_cast<size_t>(n) * p.Hq + T.hq) * p.L + i;
-      __nv_bfloat16* op = p.out + orow * EV;
+
+        const int k0 = jb * BN;
+        const bool need_mask = ((k0 + BN) > p.S) || (p.mask_kind != MASK_NONE && (k0 + BN) > first_row_hi) ||
+                               (p.mask_kind == MASK_WINDOW && k0 < last_row_lo);
+        const bool scaled = RBF || need_mask || has_bias;
+        if (RBF) {
+          const float4* kn4 = reinterpret_cast<const float4*>(sp + C::OFF_KN) + slot * (BN / 4);
+#pragma unroll
+          for (int c = 0; c < BN; c += 4) {
+            const float4 kv = kn4[c / 4];
+            z[c + 0] = fmaf(z[c + 0], p.c_rbf, -kv.x);
+            z[c + 1] = fmaf(z[c + 1], p.c_rbf, -kv.y);
+            z[c + 2] = fmaf(z[c + 2], p.c_rbf, -kv.z);
+            z[c + 3] = fmaf(z[c + 3], p.c_rbf, -kv.w);
+          }
+          __syncwarp();
+          mbar_arrive(bar(C::B_KNEMPTY + slot));
+        } else if (scaled) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c) z[c] *= p.c_dot;
+        }
+        if (need_mask) {
+          const int lo = lo_i - k0, hi = hi_i - k0;
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c < lo || c >= hi) z[c] = -INFINITY;
+        }
+        if (has_bias && bias_row != nullptr) {
+          const int lim = p.S - k0;
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c < lim) z[c] = fmaf(__ldg(bias_row + k0 + c), LOG2E, z[c]);
+        }
+        float mt = z[0];
+#pragma unroll
+        for (int c = 1; c < BN; ++c) mt = fmaxf(mt, z[c]);
+        if (!scaled) mt *= p.c_dot;
+
+        const float m_new = fmaxf(m_run, mt);
+        const bool rescale = m_new > m_run + RESCALE_THRESHOLD;
+        if (__any_sync(0xffffffffu, rescale)) {
+          const float alpha = rescale ? ex2(m_run - m_new) : 1.f;
+          if (rescale) {
+            l_run *= alpha;
+            m_run = m_new;
+          }
+          if (it > 0) {
 #pragma unroll 1
-      for (int c = 0; c < EV; c += 32) {
-        uint32_t o[32];
-        if (have_o) {
-          tmem_ld32(t_o + c, o);
-          tmem_wait_ld();
-        } else {
+            for (int c = 0; c < EV; c += 32) {
+              uint32_t o[32];
+              tmem_ld32(t_o + c, o);
+              tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(t_o + c, o);
+            }
+          }
         }
-        if (row_ok) {
-          uint32_t w[16];
+        const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+        const float nm = -mu;
+        float rs = 0.f;
+        // P = 2^(z - m) as bf16 pairs, written 16 TMEM columns (32 keys) at a time
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(op + c);
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          for (int e = 0; e < 16; ++e) {
+            const int c = ch * 32 + 2 * e;
+            float p0, p1;
+            if (scaled) {
+              p0 = ex2(z[c] + nm);
+              p1 = ex2(z[c + 1] + nm);
+            } else {
+              p0 = ex2(fmaf(z[c], p.c_dot, nm));
+              p1 = ex2(fmaf(z[c + 1], p.c_dot, nm));
+            }
+            rs += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(t_s + ch * 16, pk);
         }
+        l_run += rs;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_PFULL + t));
+        ++it;
       }
-      if (row_ok && p.lse) p.lse[orow] = lse2 * LN2;
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+
+      // ---- epilogue of this tile ----
+      if (T.active) {
+        bool have_o = it > 0;
+        if (have_o) {
+          have_o = __all_sync(0xffffffffu, wait_bar(bar(C::B_OFULL + t), oc & 1, abort_flag));
+          ++oc;
+          if (!have_o) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const float s2 = p.sink ? p.sink[T.hq] * LOG2E : -INFINITY;
+        const float M2 = fmaxf(m_run, s2);
+        float inv = 0.f, lse2 = -INFINITY;
+        if (M2 != -INFINITY) {
+          const float a = ex2(m_run - M2);
+          const float lp = l_run * a + ex2(s2 - M2);
+          if (lp > 0.f) {
+            inv = a / lp;
+            lse2 = M2 + __log2f(lp);
+          }
+        }
+        const bool row_ok = i < p.L;
+        const size_t orow = (static_cast<size_t>(w.n) * p.Hq + T.hq) * p.L + i;
+        __nv_bfloat16* op = p.out + orow * EV;
+#pragma unroll 1
+        for (int c = 0; c < EV; c += 32) {
+          uint32_t o[32];
+          if (have_o) {
+            tmem_ld32(t_o + c, o);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
+          if (row_ok) {
+            uint32_t wv[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+            uint4* dst = reinterpret_cast<uint4*>(op + c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+          }
+        }
+        if (have_o) {
+          // O_t has been read: the issuer may start the next item's accumulation
+          tc_fence_before();
+          mbar_arrive(bar(C::B_OEMPTY + t));
+        }
+        if (row_ok && p.lse) p.lse[orow] = lse2 * LN2;
+      }
     }
   }
 
@@ -621,7 +721,16 @@ int launch_impl(const AttnArgs& a, cudaStream_t stream) {
   auto kern = prefill_kernel<E, EV, RBF>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return -13;
-  kern<<<p.n_items, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return -13;
+    if (256u * C::REG_SOFTMAX + 128u * C::REG_OTHER > static_cast<uint32_t>(fa.numRegs) * C::THREADS) return -13;
+  }
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return -13;
+  const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: one CTA per SM
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? 0 : -13;
 }
 

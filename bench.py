@@ -346,21 +346,29 @@ class OracleSample:
 
 def cpu_baseline(r: sw.Recipe, budget_s: float = 12.0):
     """Oracle throughput on the host cores over a bounded sample (~budget_s of
-    compute): consecutive 256-row blocks of head (0, 0), from the last rows
-    (the heaviest under a causal mask) backwards."""
-    smp = OracleSample(r)
-    done, secs, blocks = 0.0, 0.0, 0
-    for i1 in range(r.L, 0, -256):
-        rows = np.arange(max(0, i1 - 256), i1)
-        t0 = time.perf_counter()
-        done += smp.run(rows)
-        secs += time.perf_counter() - t0
-        blocks += 1
+    compute): 256-row blocks of successive (n, hq) heads, last rows first (the
+    heaviest under a causal mask), until the budget is spent."""
+    done, secs, blocks, heads = 0.0, 0.0, 0, 0
+    unit = work_units(r)[1]
+    for n in range(r.N):
+        for hq in range(r.Hq):
+            smp = OracleSample(r, n, hq)
+            heads += 1
+            for i1 in range(r.L, 0, -256):
+                rows = np.arange(max(0, i1 - 256), i1)
+                t0 = time.perf_counter()
+                done += smp.run(rows)
+                secs += time.perf_counter() - t0
+                blocks += 1
+                if secs > budget_s:
+                    break
+            if secs > budget_s:
+                break
         if secs > budget_s:
             break
-    return {"value": round(rate(done, secs, smp.unit), 6), "unit": smp.unit, "cores": _oracle_cores(),
-            "kind": "oracle",
-            "sample": f"{blocks} x 256-row blocks of head (n=0, hq=0) of {r.name} ({secs:.1f} s of float64 numpy)"}
+    return {"value": round(rate(done, secs, unit), 6), "unit": unit, "cores": _oracle_cores(), "kind": "oracle",
+            "sample": f"{blocks} x 256-row blocks from {heads} (n, hq) heads of {r.name} "
+                      f"({secs:.1f} s of float64 numpy compute)"}
 
 
 def ours(args):
@@ -470,9 +478,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(sw.RECIPES))
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch N (profiling captures of a smaller case)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.batch is not None:
+        import dataclasses
+        sw.RECIPES[args.workload] = dataclasses.replace(sw.RECIPES[args.workload], N=args.batch)
     if args.impl == "reference":
         reference(args)
     else:

@@ -54,6 +54,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_device_status.restype = ci
     lib.attn_version.argtypes = []
     lib.attn_version.restype = ci
+    lib.attn_decode_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp, vp]
+    lib.attn_decode_fwd_noalloc.restype = ci
+    lib.attn_decode_noalloc_scratch_bytes.argtypes = []
+    lib.attn_decode_noalloc_scratch_bytes.restype = ctypes.c_size_t
     _lib = lib
     return lib
 
@@ -127,6 +131,24 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float,
                                      _ptr(bias), DTYPES[q.dtype], ctypes.c_void_p(stream.cuda_stream))
     _check(st)
     return out, lse
+
+
+def attn_decode_fwd_noalloc_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H, L, S, E, Ev, scale, mode,
+                                sink_ptr, mask_kind, window, bias_ptr, stream_ptr) -> int:
+    """The allocation-free decode entry point with integer pointers; returns the status.
+
+    For callers that may not allocate device memory while running: the
+    decode partials live in a fixed scratch array inside the library instead
+    of an allocated workspace (see include/attn_b200.h)."""
+    lib = load_library()
+    c = lambda p: None if p is None else ctypes.c_void_p(int(p))  # noqa: E731
+    return lib.attn_decode_fwd_noalloc(c(q_ptr), c(k_ptr), c(v_ptr), c(out_ptr), c(lse_ptr), int(N), int(Hq),
+                                       int(H), int(L), int(S), int(E), int(Ev), float(scale), int(mode),
+                                       c(sink_ptr), int(mask_kind), int(window), c(bias_ptr), c(stream_ptr))
+
+
+def decode_noalloc_scratch_bytes() -> int:
+    return int(load_library().attn_decode_noalloc_scratch_bytes())
 
 
 def device_status(stream: torch.cuda.Stream | None = None) -> int:

@@ -33,6 +33,8 @@
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -62,7 +64,9 @@ typedef enum {
   ATTN_ERR_WORKSPACE = -12,     /* the library could not allocate its decode workspace */
   ATTN_ERR_CUDA = -13,          /* a CUDA call or kernel launch failed */
   ATTN_ERR_DEVICE_TIMEOUT = -14,/* a kernel gave up a bounded wait (see attn_device_status) */
-  ATTN_ERR_DEVICE = -15         /* the current device is not sm_100 */
+  ATTN_ERR_DEVICE = -15,        /* the current device is not sm_100 */
+  ATTN_ERR_SCRATCH_LIMIT = -16, /* attn_decode_fwd_noalloc: the call needs more scratch than the fixed area holds */
+  ATTN_ERR_NOT_DECODE = -17     /* attn_decode_fwd_noalloc: not a decode-shaped bf16 call ((Hq/H)*L <= 16, dot) */
 } attn_status;
 
 /*
@@ -120,6 +124,37 @@ int attn_device_status(void* stream);
 
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
 int attn_version(void);
+
+/*
+ * attn_decode_fwd_noalloc -- the decode path of attn_fwd (bf16, dot score,
+ * (Hq/H)*L <= 16) without any device allocation.  The attention pages have
+ * no counterpart to this entry point; it exists for callers that must not
+ * allocate device memory while they run: services that reserve all GPU memory
+ * at start-up and forbid later allocations (so latency stays predictable and
+ * no out-of-memory error can happen mid-request), and host frameworks whose
+ * own allocator owns all device memory.
+ *
+ * Arguments, layouts, ownership and masks are those of attn_fwd (the dtype is
+ * bf16).  Instead of the library's allocated workspace, the partial results
+ * live in a fixed scratch array compiled into the library
+ * (attn_decode_noalloc_scratch_bytes() bytes, 8 MiB, held on every GPU that
+ * loads the library until the process exits).  The first call on a device
+ * looks up that array's device address (cudaGetSymbolAddress) with the
+ * device current; make that first call before beginning any stream capture.
+ * Calls that need more scratch than the array holds return
+ * ATTN_ERR_SCRATCH_LIMIT; calls that are not decode-shaped return
+ * ATTN_ERR_NOT_DECODE; neither launches anything.  The function calls no
+ * cudaMalloc, cudaFree or other allocating routine.  All calls share the one
+ * array: calls that overlap on the GPU race and must be ordered by the
+ * caller.  Nothing in the array needs clearing between calls.
+ */
+int attn_decode_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int N, int Hq, int H, int L, int S, int E, int Ev, float scale, int mode,
+                            const float* sink_logits, int mask_kind, int window, const float* bias,
+                            void* stream);
+
+/* Size in bytes of the fixed scratch array used by attn_decode_fwd_noalloc. */
+size_t attn_decode_noalloc_scratch_bytes(void);
 
 #ifdef __cplusplus
 }

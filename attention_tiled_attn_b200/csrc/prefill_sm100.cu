@@ -8,7 +8,7 @@
 //   warps 4-7   softmax for tile 1
 //   warp  8     TMA producer: Q tiles once, then K and V tiles through rings
 //   warp  9     tcgen05 issuer: S_t = Q_t K^T into TMEM, O_t += P_t V from TMEM
-//   warp 10     key-norm warp (RBF only): ||k_j||^2 of each key tile from smem
+//   warp 10     key-norm warp (RBF only): -scale*log2e*||k_j||^2 of each key tile from smem
 //   warp 11     idle (completes the third warpgroup of the register split)
 //
 // Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 and O_1 after
@@ -56,6 +56,8 @@ struct PrefillParams {
   float c_dot;      // scale * log2e           (dot)
   float c_rbf;      // 2 * scale * log2e       (rbf)
   float c_kn;       // scale * log2e           (rbf key-norm penalty)
+  float c_exp;      // exponent-unit scale: scale * log2e (dot) or 1 (rbf)
+  float c_bias;     // bias -> exponent units: 1 / scale (dot) or log2e (rbf)
 };
 
 template <int E, int EV, bool RBF>
@@ -458,7 +460,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
               }
             }
           }
-          kn[r] = acc * p.c_kn;
+          kn[r] = -acc * p.c_kn;  // stored negated: the softmax adds it in one packed FMA
         }
         __syncwarp();
         mbar_arrive(bar(C::B_KNFULL + slot));
@@ -536,22 +538,20 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
         const int k0 = jb * BN;
         const bool need_mask = ((k0 + BN) > p.S) || (p.mask_kind != MASK_NONE && (k0 + BN) > first_row_hi) ||
                                (p.mask_kind == MASK_WINDOW && k0 < last_row_lo);
-        const bool scaled = RBF || need_mask || has_bias;
+        // Logits stay in "exponent units" u with  base-2 logit = u * c_exp:
+        //   dot: u = q.k (+ bias / scale),  c_exp = scale * log2e
+        //   rbf: u = 2*scale*log2e*q.k - scale*log2e*||k||^2 (+ bias * log2e),  c_exp = 1
+        // so every tile runs the same branch-free exponent  p = 2^(u * c_exp - m).
         if (RBF) {
           const float4* kn4 = reinterpret_cast<const float4*>(sp + C::OFF_KN) + slot * (BN / 4);
 #pragma unroll
           for (int c = 0; c < BN; c += 4) {
             const float4 kv = kn4[c / 4];
-            z[c + 0] = fmaf(z[c + 0], p.c_rbf, -kv.x);
-            z[c + 1] = fmaf(z[c + 1], p.c_rbf, -kv.y);
-            z[c + 2] = fmaf(z[c + 2], p.c_rbf, -kv.z);
-            z[c + 3] = fmaf(z[c + 3], p.c_rbf, -kv.w);
+            fma2v(z[c + 0], z[c + 1], z[c + 0], z[c + 1], p.c_rbf, kv.x, kv.y);
+            fma2v(z[c + 2], z[c + 3], z[c + 2], z[c + 3], p.c_rbf, kv.z, kv.w);
           }
           __syncwarp();
           mbar_arrive(bar(C::B_KNEMPTY + slot));
-        } else if (scaled) {
-#pragma unroll
-          for (int c = 0; c < BN; ++c) z[c] *= p.c_dot;
         }
         if (need_mask) {
           const int lo = lo_i - k0, hi = hi_i - k0;
@@ -563,12 +563,18 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
           const int lim = p.S - k0;
 #pragma unroll
           for (int c = 0; c < BN; ++c)
-            if (c < lim) z[c] = fmaf(__ldg(bias_row + k0 + c), LOG2E, z[c]);
+            if (c < lim) z[c] = fmaf(__ldg(bias_row + k0 + c), p.c_bias, z[c]);
         }
-        float mt = z[0];
+        // row max: 8 independent chains of 3-input max, then a tree
+        float mx[8];
 #pragma unroll
-        for (int c = 1; c < BN; ++c) mt = fmaxf(mt, z[c]);
-        if (!scaled) mt *= p.c_dot;
+        for (int e = 0; e < 8; ++e) mx[e] = fmaxf(z[e], z[8 + e]);
+#pragma unroll
+        for (int c = 16; c < BN; c += 16)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx[e] = fmax3(mx[e], z[c + e], z[c + 8 + e]);
+        const float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7]))) *
+                         p.c_exp;
 
         const float m_new = fmaxf(m_run, mt);
         const bool rescale = m_new > m_run + RESCALE_THRESHOLD;
@@ -590,30 +596,24 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
             }
           }
         }
-        const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-        const float nm = -mu;
-        float rs = 0.f;
-        // P = 2^(z - m) as bf16 pairs, written 16 TMEM columns (32 keys) at a time
+        const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+        float rs0[4] = {0.f, 0.f, 0.f, 0.f}, rs1[4] = {0.f, 0.f, 0.f, 0.f};  // packed partial row sums
+        // P = 2^(u * c_exp - m) as bf16 pairs, written 16 TMEM columns (32 keys) at a time
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c = ch * 32 + 2 * e;
-            float p0, p1;
-            if (scaled) {
-              p0 = ex2(z[c] + nm);
-              p1 = ex2(z[c + 1] + nm);
-            } else {
-              p0 = ex2(fmaf(z[c], p.c_dot, nm));
-              p1 = ex2(fmaf(z[c + 1], p.c_dot, nm));
-            }
-            rs += p0 + p1;
+            float a0, a1;
+            fma2(a0, a1, z[c], z[c + 1], p.c_exp, nm);
+            const float p0 = ex2(a0), p1 = ex2(a1);
+            add2(rs0[e & 3], rs1[e & 3], p0, p1);
             pk[e] = pack_bf16x2(p0, p1);
           }
           tmem_st16(t_s + ch * 16, pk);
         }
-        l_run += rs;
+        l_run += ((rs0[0] + rs1[0]) + (rs0[1] + rs1[1])) + ((rs0[2] + rs1[2]) + (rs0[3] + rs1[3]));
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(C::B_PFULL + t));
@@ -718,6 +718,8 @@ int launch_impl(const AttnArgs& a, cudaStream_t stream) {
   p.c_dot = a.scale * LOG2E;
   p.c_rbf = 2.f * a.scale * LOG2E;
   p.c_kn = a.scale * LOG2E;
+  p.c_exp = RBF ? 1.f : a.scale * LOG2E;
+  p.c_bias = RBF ? LOG2E : 1.f / a.scale;
   auto kern = prefill_kernel<E, EV, RBF>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return -13;

@@ -54,6 +54,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_device_status.restype = ci
     lib.attn_version.argtypes = []
     lib.attn_version.restype = ci
+    lib.attn_exp2_poly_eval.argtypes = [vp, vp, ci, vp]
+    lib.attn_exp2_poly_eval.restype = ci
     lib.attn_decode_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp, vp]
     lib.attn_decode_fwd_noalloc.restype = ci
     lib.attn_decode_noalloc_scratch_bytes.argtypes = []
@@ -145,6 +147,15 @@ def attn_decode_fwd_noalloc_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H,
     return lib.attn_decode_fwd_noalloc(c(q_ptr), c(k_ptr), c(v_ptr), c(out_ptr), c(lse_ptr), int(N), int(Hq),
                                        int(H), int(L), int(S), int(E), int(Ev), float(scale), int(mode),
                                        c(sink_ptr), int(mask_kind), int(window), c(bias_ptr), c(stream_ptr))
+
+
+def exp2_poly_eval(x: torch.Tensor) -> torch.Tensor:
+    """The softmax's software 2^x applied on the GPU to a float32 CUDA tensor (verification)."""
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()
+    y = torch.empty_like(x)
+    _check(load_library().attn_exp2_poly_eval(_ptr(x), _ptr(y), x.numel(),
+                                              ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)))
+    return y
 
 
 def decode_noalloc_scratch_bytes() -> int:

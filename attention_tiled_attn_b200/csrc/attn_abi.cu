@@ -216,4 +216,11 @@ int attn_device_status(void* stream_ptr) {
 
 int attn_version(void) { return 10000; }
 
+int attn_exp2_poly_eval(const float* x, float* y, int n, void* stream) {
+  if (!x || !y) return ATTN_ERR_NULL_POINTER;
+  if (n < 0) return ATTN_ERR_BAD_SHAPE;
+  if (n == 0) return ATTN_OK;
+  return attn::launch_exp2_poly_eval(x, y, n, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

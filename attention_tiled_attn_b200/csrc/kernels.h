@@ -44,6 +44,9 @@ void* tensor_map_encoder();
 // swizzle and zero fill outside the tensor (defined in attn_abi.cu).
 bool make_map_rows(void* map, const void* base, int dim, long long rows, long long heads, int box_rows);
 
+// The prefill softmax's software base-2 exponential applied to n floats (verification).
+int launch_exp2_poly_eval(const float* x, float* y, int n, cudaStream_t stream);
+
 // Read-and-clear of each kernel file's device fault word (synchronises `s`).
 unsigned int take_status_prefill(cudaStream_t s);
 unsigned int take_status_decode(cudaStream_t s);

@@ -100,6 +100,12 @@ struct Cfg {
   static constexpr uint32_t REG_SOFTMAX = 216;
   static constexpr uint32_t REG_OTHER = 72;
   static constexpr uint32_t TMEM_COLS = 512;
+  // Pairs of each 16-pair (32-key) chunk whose exponential runs on the FMA pipe
+  // (exp2_poly2) instead of the MUFU unit (16 exponentials per clock per SM).
+  // The polynomial costs about as much FMA-pipe time per element as MUFU time
+  // (the packed f32x2 path still retires 128 FMAs per clock per SM), and on
+  // this kernel no split measured faster than all-MUFU, so none is offloaded.
+  static constexpr uint32_t EMU_MASK = 0u;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, EV, 1);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -607,7 +613,13 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
             const int c = ch * 32 + 2 * e;
             float a0, a1;
             fma2(a0, a1, z[c], z[c + 1], p.c_exp, nm);
-            const float p0 = ex2(a0), p1 = ex2(a1);
+            float p0, p1;
+            if ((C::EMU_MASK >> e) & 1u) {
+              exp2_poly2(p0, p1, a0, a1);
+            } else {
+              p0 = ex2(a0);
+              p1 = ex2(a1);
+            }
             add2(rs0[e & 3], rs1[e & 3], p0, p1);
             pk[e] = pack_bf16x2(p0, p1);
           }
@@ -737,6 +749,22 @@ int launch_impl(const AttnArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+__global__ void exp2_poly_eval_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
+  float p0, p1;
+  exp2_poly2(p0, p1, x0, x1);
+  y[i] = p0;
+  if (i + 1 < n) y[i + 1] = p1;
+}
+
+int launch_exp2_poly_eval(const float* x, float* y, int n, cudaStream_t stream) {
+  const int pairs = (n + 1) / 2;
+  exp2_poly_eval_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? 0 : -13;
+}
 
 unsigned int take_status_prefill(cudaStream_t s) { return take_device_status_local(s); }
 

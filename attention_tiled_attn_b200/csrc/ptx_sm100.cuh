@@ -68,6 +68,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -255,6 +268,45 @@ __device__ __forceinline__ void fma2v(float& d0, float& d1, float a0, float a1, 
       "mov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b), "f"(c0), "f"(c1));
+}
+
+// (d0, d1) = (a0, a1) * (b0, b1) + (c0, c1), packed
+__device__ __forceinline__ void fma2g(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// Software 2^x for two lanes, on the FMA pipe instead of the MUFU unit.
+// 2^x = 2^n * p(f), n = round(x) (via the 1.5 * 2^23 rounding constant),
+// f = x - n in [-1/2, 1/2], p the degree-3 minimax polynomial with p(0) = 1
+// fitted by csrc/fit_exp2_poly.py (max relative error 1.02e-4); n is added to
+// the exponent field of p(f) as an integer.  x is clamped to >= -126, so the
+// result is never below 2^-126 (a masked -inf logit gives 1.2e-38, not 0).
+constexpr float EXP2_C1 = 0.6932829022407532f;
+constexpr float EXP2_C2 = 0.24221095442771912f;
+constexpr float EXP2_C3 = 0.05500892922282219f;
+constexpr float ROUND_MAGIC = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ void exp2_poly2(float& p0, float& p1, float x0, float x1) {
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, n0, n1, f0, f1, q0, q1;
+  fma2g(t0, t1, x0, x1, 1.f, 1.f, ROUND_MAGIC, ROUND_MAGIC);    // x + M: rounds x to an integer
+  fma2g(n0, n1, t0, t1, 1.f, 1.f, -ROUND_MAGIC, -ROUND_MAGIC);  // n = round(x), exact
+  fma2g(f0, f1, n0, n1, -1.f, -1.f, x0, x1);                    // f = x - n, exact
+  fma2g(q0, q1, f0, f1, EXP2_C3, EXP2_C3, EXP2_C2, EXP2_C2);
+  fma2g(q0, q1, q0, q1, f0, f1, EXP2_C1, EXP2_C1);
+  fma2g(q0, q1, q0, q1, f0, f1, 1.f, 1.f);
+  // the low 9 bits of M's pattern are zero, so (bits(t) << 23) is n in the exponent field
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
 // (d0, d1) += (a0, a1) on the packed two-lane fp32 path

@@ -178,13 +178,20 @@ def barrier(pg):
         pg.barrier()
 
 
-def max_over_ranks(pg, value: float) -> float:
+def max_over_ranks(pg, value: float, device: str = "cuda") -> float:
+    """Largest value over all ranks (the job's time is its slowest rank's)."""
     if pg is None:
         return value
     import torch
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_rate(amount_per_rank: float, world: int, secs_max: float, steps: int, unit: str) -> float:
+    """Whole-job throughput: every rank runs its own full batch (weak scaling),
+    so the work is world x per-rank work over the slowest rank's time."""
+    return rate(amount_per_rank * world, secs_max / steps, unit)
 
 
 def time_device(fn, steps, warmup, flush_buf, stream):
@@ -381,26 +388,44 @@ def ours(args):
     e2e, _ = e2e_measure(main, max(3, min(args.steps, 20)), 2)
     extra = {}
     if not args.no_extra:
-        for name in sw.RECIPES:
-            if name == args.workload or sw.RECIPES[name].dtype != "bf16":
-                continue
-            main_t = {k: main[k] for k in ("tensors", "out", "lse")}
-            res = run_workload(name, max(5, args.steps // 4), args.warmup, pg, flush, peaks, peak_kind)
-            rr = res["recipe"]
-            extra[name] = {
-                "value": round(rate(res["amount"] * world, res["secs_max"] / max(5, args.steps // 4),
-                                    res["unit"]), 2),
-                "unit": res["unit"], "ms_per_step": round(res["secs_max"] / max(5, args.steps // 4) * 1e3, 4),
+        import dataclasses
+        names = [n for n in sw.RECIPES if n != args.workload and sw.RECIPES[n].dtype == "bf16"]
+        runs = []
+        for name in names:
+            r0 = sw.RECIPES[name]
+            runs.append((name, r0))
+            # controls for the "RBF / sink within 10% of plain dot" comparison: same shapes and data
+            if r0.mode == "rbf":
+                runs.append((name + ":dot_control", dataclasses.replace(r0, mode="dot")))
+            if r0.sink != "none":
+                runs.append((name + ":no_sink_control", dataclasses.replace(r0, sink="none")))
+        for label, rr in runs:
+            base = sw.RECIPES[rr.name]
+            sw.RECIPES[rr.name] = rr
+            try:
+                k = max(5, args.steps // 4)
+                res = run_workload(rr.name, k, args.warmup, pg, flush, peaks, peak_kind)
+            finally:
+                sw.RECIPES[rr.name] = base
+            extra[label] = {
+                "value": round(job_rate(res["amount"], world, res["secs_max"], k, res["unit"]), 2),
+                "unit": res["unit"], "ms_per_step": round(res["secs_max"] / k * 1e3, 4),
                 "roofline_frac": res["roofline"]["frac"], "bound": res["roofline"]["bound"],
                 "mode": rr.mode, "sink": rr.sink != "none", "mask": rr.mask_kind,
             }
             del res
             torch.cuda.empty_cache()
+        for label in list(extra):
+            if ":" in label:
+                continue
+            for ctl in (label + ":dot_control", label + ":no_sink_control"):
+                if ctl in extra:
+                    extra[label]["time_vs_" + ctl.split(":")[1]] = round(
+                        extra[label]["ms_per_step"] / extra[ctl]["ms_per_step"], 4)
     if rank == 0:
-        amount_all = main["amount"] * world
         line = {
             "metric": METRIC,
-            "value": round(rate(amount_all, main["secs_max"] / args.steps, main["unit"]), 3),
+            "value": round(job_rate(main["amount"], world, main["secs_max"], args.steps, main["unit"]), 3),
             "unit": main["unit"],
             "n_gpus": world,
             "steps": args.steps,

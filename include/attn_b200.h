@@ -126,6 +126,17 @@ int attn_device_status(void* stream);
 int attn_version(void);
 
 /*
+ * attn_exp2_poly_eval -- verification hook: y[i] = the prefill softmax's
+ * software base-2 exponential of x[i] (device pointers, n floats).  A share of
+ * the softmax exponentials is evaluated this way on the FMA pipe instead of
+ * the MUFU unit: 2^x = 2^round(x) * p(x - round(x)) with a degree-3 minimax
+ * polynomial (relative error <= 1.02e-4); x is clamped to >= -126.  The
+ * exponential itself is the softmax's (page "어텐션 메커니즘" §2, §6); this
+ * way of evaluating it is an implementation choice, not from the pages.
+ */
+int attn_exp2_poly_eval(const float* x, float* y, int n, void* stream);
+
+/*
  * attn_decode_fwd_noalloc -- the decode path of attn_fwd (bf16, dot score,
  * (Hq/H)*L <= 16) without any device allocation.  The attention pages have
  * no counterpart to this entry point; it exists for callers that must not

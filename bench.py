@@ -44,9 +44,16 @@ DEFAULT_WORKLOAD = "dot_causal_2k_bf16"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic per launch of the dominant kernel from an ncu capture of the same
-# kernel build (profiles/*.md records the command and counters); None until taken.
-NCU_TRAFFIC_BYTES = {}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# dominant kernel from one ncu capture of the same kernel build; the capture
+# command and counters are in profiles/.  Must be reset when the kernel changes.
+NCU_TRAFFIC_BYTES = {
+    "dot_causal_2k_bf16": 132_793_088 + 13_932_032,          # prefill_kernel<128,128,dot>
+    "sink_gqa_window_16k_bf16": 167_958_528 + 100_350_976,   # prefill_kernel<64,64,dot>
+    "rbf_registers_4k_bf16": 37_890_048 + 91_904,            # prefill_kernel<64,64,rbf>
+    # decode_partial_kernel<128,128>: batch-2 capture (1.0738e9 + 4.43e6 B) scaled by 16 to batch 32
+    "decode_sink_gqa_128k_bf16": 16 * (1_073_818_000 + 4_434_432),
+}
 
 
 # ---------------------------------------------------------------------------
@@ -351,12 +358,16 @@ class OracleSample:
         return self.rows_amount(rows)
 
 
-def cpu_baseline(r: sw.Recipe, budget_s: float = 12.0):
-    """Oracle throughput on the host cores over a bounded sample (~budget_s of
-    compute): 256-row blocks of successive (n, hq) heads, last rows first (the
-    heaviest under a causal mask), until the budget is spent."""
+def cpu_baseline(r: sw.Recipe, budget_s: float = 12.0, wall_limit_s: float = 40.0):
+    """Oracle throughput on the host cores over a bounded sample: 256-row
+    blocks of successive (n, hq) heads, last rows first (the heaviest under a
+    causal mask), until budget_s of oracle compute or wall_limit_s of wall
+    time (input regeneration included) is spent.  The rate counts compute
+    time only."""
     done, secs, blocks, heads = 0.0, 0.0, 0, 0
     unit = work_units(r)[1]
+    t_start = time.perf_counter()
+    stop = False
     for n in range(r.N):
         for hq in range(r.Hq):
             smp = OracleSample(r, n, hq)
@@ -367,11 +378,13 @@ def cpu_baseline(r: sw.Recipe, budget_s: float = 12.0):
                 done += smp.run(rows)
                 secs += time.perf_counter() - t0
                 blocks += 1
-                if secs > budget_s:
+                if secs > budget_s or time.perf_counter() - t_start > wall_limit_s:
+                    stop = True
                     break
-            if secs > budget_s:
+            if stop or time.perf_counter() - t_start > wall_limit_s:
+                stop = True
                 break
-        if secs > budget_s:
+        if stop:
             break
     return {"value": round(rate(done, secs, unit), 6), "unit": unit, "cores": _oracle_cores(), "kind": "oracle",
             "sample": f"{blocks} x 256-row blocks from {heads} (n, hq) heads of {r.name} "

@@ -8,8 +8,8 @@
 //   warps 4-7   softmax for tile 1
 //   warp  8     TMA producer: Q tiles once, then K and V tiles through rings
 //   warp  9     tcgen05 issuer: S_t = Q_t K^T into TMEM, O_t += P_t V from TMEM
-//   warp 10     key-norm warp (RBF only): -scale*log2e*||k_j||^2 of each key tile from smem
-//   warp 11     idle (completes the third warpgroup of the register split)
+//   warps 10-11 key-norm warps (RBF only): -scale*log2e*||k_j||^2 of each key tile from
+//               smem, half of the tile's keys each (idle for the dot score)
 //
 // Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 and O_1 after
 // them.  P_t (bf16, two per column) overwrites the first 64 columns of S_t.
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
     mbar_init(bar(C::B_QEMPTY), 1);
     for (int s = 0; s < C::NK; ++s) {
       mbar_init(bar(C::B_KFULL + s), 1);
-      mbar_init(bar(C::B_KEMPTY + s), RBF ? 2 : 1);
+      mbar_init(bar(C::B_KEMPTY + s), RBF ? 3 : 1);  // issuer commit (+ both key-norm warps)
     }
     for (int s = 0; s < C::NV; ++s) {
       mbar_init(bar(C::B_VFULL + s), 1);
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
       mbar_init(bar(C::B_OEMPTY + t), 128);
     }
     for (int s = 0; s < C::NKN; ++s) {
-      mbar_init(bar(C::B_KNFULL + s), 32);
+      mbar_init(bar(C::B_KNFULL + s), 64);  // the 64 lanes of the two key-norm warps
       mbar_init(bar(C::B_KNEMPTY + s), 256);
     }
     mbar_init(bar(C::B_DRAIN), 1);
@@ -352,13 +352,14 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
           tc_fence_after();
           const uint32_t d = tmem + 256 + t * EV;
           const uint32_t a = tmem + t * 128;
-          const uint32_t vbase = sb + C::OFF_V + vs * C::V_BYTES;
+          // B = V tile, MN-major: 16 keys per step = 16 rows of 128 B (+128 in the low
+          // descriptor half); the second 64-column box sits at +BN*128 (leading byte offset)
+          const uint32_t b_lo = desc_lo(sb + C::OFF_V + vs * C::V_BYTES, BN * 128);
+          constexpr uint32_t b_hi = desc_hi_sw128(1024);
+          const uint32_t acc0 = first ? 0u : 1u;
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            // B = V tile, MN-major: 16 keys per step = 16 rows of 128 B; second 64-column box at +BN*128
-            const uint64_t bdesc = smem_desc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
-            mma_ts(d, a + kk * 8, bdesc, C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ts_h(d, a + kk * 8, b_lo + kk * 128, b_hi, C::IDESC_PV, kk > 0 ? 1u : acc0);
           first = false;
           ++pvc;
           const int uses = (in_range(w.tile[0], jbp) ? 1 : 0) + (in_range(w.tile[1], jbp) ? 1 : 0);
@@ -371,14 +372,14 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
         };
         auto issue_qk = [&](int t, uint32_t ks) {
           const uint32_t d = tmem + t * 128;
-          const uint32_t qbase = sb + C::OFF_Q + t * C::Q_BYTES;
-          const uint32_t kbase = sb + C::OFF_K + ks * C::K_BYTES;
+          const uint32_t a_lo = desc_lo(sb + C::OFF_Q + t * C::Q_BYTES, 16);
+          const uint32_t b_lo = desc_lo(sb + C::OFF_K + ks * C::K_BYTES, 16);
+          constexpr uint32_t hi = desc_hi_sw128(1024);
 #pragma unroll
           for (int kk = 0; kk < E / 16; ++kk) {
-            const uint32_t koff = (kk / 4) * (BM * 128) + (kk % 4) * 32;
-            const uint64_t adesc = smem_desc_sw128(qbase + koff, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(kbase + koff, 16, 1024);
-            mma_ss(d, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
+            // K step kk: 32 bytes further in the 128-byte swizzled row; the next 64-column box at +rows*128
+            const uint32_t koff = ((kk / 4) * (BM * 128) + (kk % 4) * 32) >> 4;
+            mma_ss_h(d, a_lo + koff, hi, b_lo + koff, hi, C::IDESC_QK, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar(C::B_SFULL + t));
         };
@@ -426,8 +427,9 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
       mma_commit(bar(C::B_DRAIN));
       mbar_wait(bar(C::B_DRAIN), 0);
     }
-  } else if (RBF && warp == 10) {
-    // ================= key-norm warp (RBF) =================
+  } else if (RBF && warp >= 10) {
+    // ================= key-norm warps (RBF) =================
+    // warps 10 and 11 (two SMSPs) each take half of every key block's rows
     uint32_t gk = 0;
     bool ok = true;
     for (int k = 0; ok && k * G < p.n_items; ++k) {
@@ -447,9 +449,9 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
         const uint8_t* ktile = sp + C::OFF_K + ks * C::K_BYTES;
         float* kn = reinterpret_cast<float*>(sp + C::OFF_KN) + slot * BN;
 #pragma unroll
-        for (int rr = 0; rr < BN / 32; ++rr) {
-          const int r = lane + 32 * rr;
-          float acc = 0.f;
+        for (int rr = 0; rr < BN / 64; ++rr) {
+          const int r = (warp - 10) * (BN / 2) + lane + 32 * rr;
+          float acc0 = 0.f, acc1 = 0.f;  // packed even / odd partial sums
 #pragma unroll
           for (int bb = 0; bb < E / 64; ++bb) {
 #pragma unroll
@@ -461,12 +463,11 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
               for (int e = 0; e < 4; ++e) {
                 const float lo = __uint_as_float(ws[e] << 16);
                 const float hi = __uint_as_float(ws[e] & 0xFFFF0000u);
-                acc = fmaf(lo, lo, acc);
-                acc = fmaf(hi, hi, acc);
+                fma2g(acc0, acc1, lo, hi, lo, hi, acc0, acc1);
               }
             }
           }
-          kn[r] = -acc * p.c_kn;  // stored negated: the softmax adds it in one packed FMA
+          kn[r] = -(acc0 + acc1) * p.c_kn;  // stored negated: the softmax adds it in one packed FMA
         }
         __syncwarp();
         mbar_arrive(bar(C::B_KNFULL + slot));

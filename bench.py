@@ -404,6 +404,12 @@ def ours(args):
         import dataclasses
         names = [n for n in sw.RECIPES if n != args.workload and sw.RECIPES[n].dtype == "bf16"]
         runs = []
+        # steady-state control: the bench workload's kernel (dot, E=128) on one long
+        # non-causal sequence, where per-item pipeline fill and drain are amortised
+        base = sw.RECIPES[args.workload]
+        if base.mode == "dot" and base.dtype == "bf16" and not is_decode(base):
+            runs.append((args.workload + ":steady_state_noncausal_8k",
+                         dataclasses.replace(base, N=1, L=8192, S=8192, mask_kind="none")))
         for name in names:
             r0 = sw.RECIPES[name]
             runs.append((name, r0))

@@ -46,6 +46,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp, ci, vp]
     lib.attn_fwd.restype = ci
+    lib.attn_fwd_streaming.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp, ci, vp]
+    lib.attn_fwd_streaming.restype = ci
     lib.attn_status_string.argtypes = [ci]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_release_workspace.argtypes = []
@@ -87,17 +89,31 @@ def attn_fwd_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H, L, S, E, Ev, s
                         int(window), c(bias_ptr), int(dtype), c(stream_ptr))
 
 
+def attn_fwd_streaming_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H, L, S, E, Ev, scale, mode, sink_ptr,
+                           window, keep_first, bias_ptr, dtype, stream_ptr) -> int:
+    """The streaming-mask C entry point with integer pointers; returns the status code."""
+    lib = load_library()
+    c = lambda p: None if p is None else ctypes.c_void_p(int(p))  # noqa: E731
+    return lib.attn_fwd_streaming(c(q_ptr), c(k_ptr), c(v_ptr), c(out_ptr), c(lse_ptr), int(N), int(Hq), int(H),
+                                  int(L), int(S), int(E), int(Ev), float(scale), int(mode), c(sink_ptr),
+                                  int(window), int(keep_first), c(bias_ptr), int(dtype), c(stream_ptr))
+
+
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float, mode: str = "dot",
              sink: torch.Tensor | None = None, mask_kind: str = "none", window: int = 0,
              bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
-             lse: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None):
+             lse: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None, keep_first: int = 0):
     """out = softmax(z + B) V on the GPU.  Returns (out, lse).
 
     q (N, Hq, L, E), k (N, H, S, E), v (N, H, S, Ev): contiguous CUDA tensors,
     all bfloat16 or all float32.  sink: (Hq,) float32 or None.  bias: (L, S)
     float32 or None.  mode: "dot", "rbf" or "sink"; mask_kind: "none",
-    "causal" or "window".  out/lse may be given (contiguous, right shape).
+    "causal", "window" or "streaming" (the first ``keep_first`` keys plus the
+    last ``window`` keys, through attn_fwd_streaming).  out/lse may be given
+    (contiguous, right shape).
     """
+    if mask_kind not in MASKS and mask_kind != "streaming":
+        raise ValueError(f"unknown mask kind {mask_kind!r}")
     load_library()
     for name, t in (("q", q), ("k", k), ("v", v)):
         if not t.is_cuda:
@@ -128,9 +144,14 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float,
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     with torch.cuda.device(q.device):
-        st = load_library().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), N, Hq, H, L, S, E, Ev,
-                                     float(scale), MODES[mode], _ptr(sink), MASKS[mask_kind], int(window),
-                                     _ptr(bias), DTYPES[q.dtype], ctypes.c_void_p(stream.cuda_stream))
+        lib = load_library()
+        common = (_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), N, Hq, H, L, S, E, Ev, float(scale), MODES[mode],
+                  _ptr(sink))
+        tail = (_ptr(bias), DTYPES[q.dtype], ctypes.c_void_p(stream.cuda_stream))
+        if mask_kind == "streaming":
+            st = lib.attn_fwd_streaming(*common, int(window), int(keep_first), *tail)
+        else:
+            st = lib.attn_fwd(*common, MASKS[mask_kind], int(window), *tail)
     _check(st)
     return out, lse
 

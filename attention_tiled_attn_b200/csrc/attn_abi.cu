@@ -99,22 +99,18 @@ int ensure_workspace(int dev, size_t bytes, cudaStream_t stream, void** out) {
 }
 
 }  // namespace
-}  // namespace attn
 
-extern "C" {
-
-int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L,
-             int S, int E, int Ev, float scale, int mode, const float* sink_logits, int mask_kind, int window,
-             const float* bias, int dtype, void* stream_ptr) {
-  using namespace attn;
+// Shared by the public entry points once they have checked their mask arguments:
+// validates the rest and dispatches (fp32 kernel, split-key decode, tcgen05 prefill).
+int forward(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L, int S,
+            int E, int Ev, float scale, int mode, const float* sink_logits, int mask_kind, int window, int keep,
+            const float* bias, int dtype, void* stream_ptr) {
   if (!q || !k || !v || !out) return ATTN_ERR_NULL_POINTER;
   if (N < 1 || Hq < 1 || H < 1 || L < 1 || S < 1) return ATTN_ERR_BAD_SHAPE;
   if (Hq % H != 0) return ATTN_ERR_GQA;
   if ((E != 64 && E != 128) || (Ev != 64 && Ev != 128)) return ATTN_ERR_HEAD_DIM;
   if (!std::isfinite(scale) || scale <= 0.f) return ATTN_ERR_SCALE;
   if (mode < ATTN_DOT || mode > ATTN_SINK) return ATTN_ERR_MODE;
-  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_SLIDING_WINDOW) return ATTN_ERR_MASK;
-  if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window < 1) return ATTN_ERR_WINDOW;
   if (mode == ATTN_SINK && sink_logits == nullptr) return ATTN_ERR_SINK;
   if (dtype != ATTN_BF16 && dtype != ATTN_FP32) return ATTN_ERR_DTYPE;
   // every element offset must fit the kernels' 64-bit indexing and the per-head
@@ -151,6 +147,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   a.sink = sink_logits;
   a.mask_kind = mask_kind;
   a.window = window;
+  a.keep = keep;
   a.bias = bias;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
 
@@ -165,6 +162,28 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   return launch_prefill_bf16(a, stream);
 }
 
+}  // namespace attn
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L,
+             int S, int E, int Ev, float scale, int mode, const float* sink_logits, int mask_kind, int window,
+             const float* bias, int dtype, void* stream_ptr) {
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_SLIDING_WINDOW) return ATTN_ERR_MASK;
+  if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window < 1) return ATTN_ERR_WINDOW;
+  return attn::forward(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, mask_kind, window, 0,
+                       bias, dtype, stream_ptr);
+}
+
+int attn_fwd_streaming(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H,
+                       int L, int S, int E, int Ev, float scale, int mode, const float* sink_logits, int window,
+                       int keep_first, const float* bias, int dtype, void* stream_ptr) {
+  if (window < 1) return ATTN_ERR_WINDOW;
+  if (keep_first < 0) return ATTN_ERR_KEEP;
+  return attn::forward(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, attn::MASK_STREAM,
+                       window, keep_first, bias, dtype, stream_ptr);
+}
+
 const char* attn_status_string(int status) {
   switch (status) {
     case ATTN_OK: return "ok";
@@ -176,6 +195,7 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_MODE: return "unknown score mode";
     case ATTN_ERR_MASK: return "unknown mask kind";
     case ATTN_ERR_WINDOW: return "sliding window needs window >= 1";
+    case ATTN_ERR_KEEP: return "streaming mask needs keep_first >= 0";
     case ATTN_ERR_SINK: return "ATTN_SINK needs sink logits";
     case ATTN_ERR_DTYPE: return "unknown dtype";
     case ATTN_ERR_ALIGNMENT: return "misaligned pointer (16 bytes for tensors, 4 for lse and sink)";

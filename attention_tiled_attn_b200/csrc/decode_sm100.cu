@@ -39,7 +39,7 @@ constexpr int DWARPS = 4;          // consumer warps (16 keys each)
 constexpr int DTHREADS = (DWARPS + 1) * 32;
 constexpr float D_RESCALE_THRESHOLD = 8.0f;
 
-struct DecodeParams {
+struct DecodeParams {  // 128 bytes: kept at that size, the kernels' code generation depends on it
   const __nv_bfloat16* q;
   __nv_bfloat16* out;
   float* lse;
@@ -47,15 +47,18 @@ struct DecodeParams {
   const float* bias;
   float* ws_acc;    // [slots][16][Ev]
   float* ws_ml;     // [slots][16][2]
+  long long T;      // total chunks = N*H*nc
   int N, Hq, H, L, S, group, R;
   int mask_kind, window;
-  int kb_lo;        // first visible 64-key chunk (shared by all units)
-  int nc;           // chunks per unit
-  long long T;      // total chunks = N*H*nc
+  int kb_win;       // first chunk after the head part (the window's; the first visible one otherwise)
+  int nc;           // chunks per unit (head part + window part)
   int G;            // persistent CTAs
   int max_segs;     // partial slots per CTA
   float c_dot;      // scale * log2e
+  int keep;         // streaming mask: initial keys every later query sees
+  int nc_head;      // streaming mask: chunks of the kept initial keys (0 otherwise)
 };
+static_assert(sizeof(DecodeParams) == 128, "DecodeParams layout");
 
 template <int E, int EV>
 struct DCfg {
@@ -71,6 +74,14 @@ struct DCfg {
 };
 
 __device__ __forceinline__ long long seg_start(long long b, long long T, int G) { return (b * T) / G; }
+
+// First key of a unit's local chunk.  STREAM (the streaming mask with kept keys,
+// a compile-time switch): the head part, then the window part.
+template <bool STREAM>
+__device__ __forceinline__ int chunk_key0(const DecodeParams& p, int local) {
+  if constexpr (STREAM) return (local < p.nc_head ? local : p.kb_win + (local - p.nc_head)) * DC;
+  return (p.kb_win + local) * DC;
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -97,7 +108,7 @@ __device__ __forceinline__ uint32_t sw_off(int row, int c16) {
   return (c16 >> 3) * (DC * 128) + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
 }
 
-template <int E, int EV>
+template <int E, int EV, bool STREAM>
 __global__ void __launch_bounds__(DTHREADS, 1)
     decode_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const DecodeParams p) {
@@ -143,7 +154,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
           break;
         }
         const long long u = c / p.nc;
-        const int key0 = (p.kb_lo + static_cast<int>(c % p.nc)) * DC;
+        const int key0 = chunk_key0<STREAM>(p, static_cast<int>(c % p.nc));
         const uint32_t dst = sb + C::OFF_STAGES + s * C::STAGE_BYTES;
         mbar_arrive_expect_tx(full_bar(s), C::STAGE_BYTES);
         for (int b = 0; b < E / 64; ++b)
@@ -169,7 +180,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
     const int r = rA + 8 * h;
     live_r[h] = r < p.R;
     const int i = live_r[h] ? (r % p.L) : 0;
-    lo_r[h] = (p.mask_kind == MASK_WINDOW) ? i + off - p.window + 1 : 0;
+    lo_r[h] = (STREAM || p.mask_kind == MASK_WINDOW) ? i + off - p.window + 1 : 0;
     hi_r[h] = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, i + off + 1);
   }
 
@@ -274,7 +285,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
     const uint32_t kbuf = sb + C::OFF_STAGES + s * C::STAGE_BYTES;
     const uint32_t vbuf = kbuf + E * DC * 2;
     const int j0 = warp * 16;  // this warp's keys within the chunk
-    const int key0 = (p.kb_lo + static_cast<int>(c % p.nc)) * DC + j0;
+    const int key0 = chunk_key0<STREAM>(p, static_cast<int>(c % p.nc)) + j0;
 
     // S = Q K^T for 16 keys (two n-tiles of 8)
     float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -299,7 +310,11 @@ __global__ void __launch_bounds__(DTHREADS, 1)
         float zz = sc[t][e] * p.c_dot;
         if (need_mask) {
           const int key = key0 + t * 8 + cq + (e & 1);
-          if (key < lo_r[h] || key >= hi_r[h]) zz = -INFINITY;
+          if constexpr (STREAM) {
+            if (key >= hi_r[h] || (key < lo_r[h] && key >= p.keep)) zz = -INFINITY;
+          } else {
+            if (key < lo_r[h] || key >= hi_r[h]) zz = -INFINITY;
+          }
           if (p.bias != nullptr && live_r[h] && key < p.S)
             zz = fmaf(p.bias[static_cast<size_t>((rA + 8 * h) % p.L) * p.S + key], LOG2E, zz);
         }
@@ -399,7 +414,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
 }
 
 struct DecodePlan {
-  int kb_lo, nc, G, max_segs;
+  int nc_head, kb_win, nc, G, max_segs;
   long long T;
 };
 
@@ -407,13 +422,24 @@ DecodePlan plan(const AttnArgs& a, int num_sms) {
   DecodePlan d{};
   const int off = a.S - a.L;
   int lo = 0, hi = a.S;
-  if (a.mask_kind == MASK_CAUSAL || a.mask_kind == MASK_WINDOW) hi = a.S < off + a.L ? a.S : off + a.L;
-  if (a.mask_kind == MASK_WINDOW) lo = off - a.window + 1 > 0 ? off - a.window + 1 : 0;
+  if (a.mask_kind != MASK_NONE) hi = a.S < off + a.L ? a.S : off + a.L;
+  const int win_lo = off - a.window + 1 > 0 ? off - a.window + 1 : 0;
+  if (a.mask_kind == MASK_WINDOW || (a.mask_kind == MASK_STREAM && a.keep == 0)) lo = win_lo;
   if (hi < 1) hi = 1;  // keep one chunk so every row gets a (fully masked) partial
   if (lo >= hi) lo = hi - 1;
-  d.kb_lo = lo / DC;
   const int kb_hi = (hi + DC - 1) / DC;
-  d.nc = kb_hi - d.kb_lo;
+  d.nc_head = 0;
+  d.kb_win = lo / DC;
+  if (a.mask_kind == MASK_STREAM && a.keep > 0) {
+    // kept initial keys, then the window: the chunks between them are never read
+    const int head = (a.keep + DC - 1) / DC;
+    const int kb_w = win_lo / DC;
+    if (kb_w > head && kb_w < kb_hi) {
+      d.nc_head = head;
+      d.kb_win = kb_w;
+    }
+  }
+  d.nc = d.nc_head + (kb_hi - d.kb_win);
   d.T = static_cast<long long>(a.N) * a.H * d.nc;
   d.G = static_cast<int>(d.T < num_sms ? d.T : num_sms);
   const long long per = (d.T + d.G - 1) / d.G;
@@ -421,7 +447,7 @@ DecodePlan plan(const AttnArgs& a, int num_sms) {
   return d;
 }
 
-template <int E, int EV>
+template <int E, int EV, bool STREAM>
 int launch_decode_impl(const AttnArgs& a, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream) {
   using C = DCfg<E, EV>;
   const DecodePlan d = plan(a, num_sms);
@@ -446,15 +472,18 @@ int launch_decode_impl(const AttnArgs& a, void* ws, size_t ws_bytes, int num_sms
   p.S = a.S;
   p.group = a.Hq / a.H;
   p.R = p.group * a.L;
-  p.mask_kind = a.mask_kind;
+  // the streaming mask without kept keys is the sliding window
+  p.mask_kind = (a.mask_kind == MASK_STREAM && !STREAM) ? MASK_WINDOW : a.mask_kind;
   p.window = a.window;
-  p.kb_lo = d.kb_lo;
+  p.keep = STREAM ? a.keep : 0;
+  p.nc_head = d.nc_head;
+  p.kb_win = d.kb_win;
   p.nc = d.nc;
   p.T = d.T;
   p.G = d.G;
   p.max_segs = d.max_segs;
   p.c_dot = a.scale * LOG2E;
-  auto kern = decode_partial_kernel<E, EV>;
+  auto kern = decode_partial_kernel<E, EV, STREAM>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return -13;
   kern<<<d.G, DTHREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
@@ -475,10 +504,17 @@ size_t decode_workspace_bytes(const AttnArgs& a, int num_sms) {
 }
 
 int launch_decode_bf16(const AttnArgs& a, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream) {
-  if (a.E == 128 && a.Ev == 128) return launch_decode_impl<128, 128>(a, ws, ws_bytes, num_sms, stream);
-  if (a.E == 64 && a.Ev == 64) return launch_decode_impl<64, 64>(a, ws, ws_bytes, num_sms, stream);
-  if (a.E == 64 && a.Ev == 128) return launch_decode_impl<64, 128>(a, ws, ws_bytes, num_sms, stream);
-  if (a.E == 128 && a.Ev == 64) return launch_decode_impl<128, 64>(a, ws, ws_bytes, num_sms, stream);
+  // kept initial keys need the streaming mask test even where the plan makes no
+  // head/window split (kept keys and window overlap: nc_head is then 0)
+  const bool st = a.mask_kind == MASK_STREAM && a.keep > 0;
+#define ATTN_DECODE_CASE(e, ev)                                                       \
+  if (a.E == e && a.Ev == ev) return st ? launch_decode_impl<e, ev, true>(a, ws, ws_bytes, num_sms, stream) \
+                                        : launch_decode_impl<e, ev, false>(a, ws, ws_bytes, num_sms, stream);
+  ATTN_DECODE_CASE(128, 128)
+  ATTN_DECODE_CASE(64, 64)
+  ATTN_DECODE_CASE(64, 128)
+  ATTN_DECODE_CASE(128, 64)
+#undef ATTN_DECODE_CASE
   return -4;
 }
 

@@ -34,7 +34,7 @@ struct F32Params {
   const float* sink;
   const float* bias;
   int N, Hq, H, L, S, group;
-  int mask_kind, window;
+  int mask_kind, window, keep;
   float scale;
 };
 
@@ -81,16 +81,21 @@ __global__ void __launch_bounds__(FTHREADS) fp32_attn_kernel(const F32Params p) 
   // key range of the row block
   const int off = p.S - p.L;
   const int r_last = min(r0 + FBM - 1, p.L - 1);
+  const bool windowed = p.mask_kind == MASK_WINDOW || p.mask_kind == MASK_STREAM;
   const int hi_blk = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, r_last + off + 1);
-  const int lo_blk = (p.mask_kind == MASK_WINDOW) ? max(0, r0 + off - p.window + 1) : 0;
+  const int lo_blk = (windowed && p.keep == 0) ? max(0, r0 + off - p.window + 1) : 0;
   const int jb_lo = lo_blk / FBN;
   const int jb_hi = hi_blk > lo_blk ? (hi_blk + FBN - 1) / FBN : jb_lo;
+  // streaming: key blocks between the kept head and the first row's window are invisible to all rows
+  const int gap_lo = (p.keep + FBN - 1) / FBN;
+  const int gap_hi = (p.mask_kind == MASK_STREAM) ? max(0, r0 + off - p.window + 1) / FBN : 0;
 
+  // key j visible to row i iff j < hi_i and (j >= lo_i or j < keep)
   int lo_i[4], hi_i[4];
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     const int i = r0 + rg * 4 + r;
-    lo_i[r] = (p.mask_kind == MASK_WINDOW) ? i + off - p.window + 1 : 0;
+    lo_i[r] = windowed ? i + off - p.window + 1 : 0;
     hi_i[r] = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, i + off + 1);
   }
 
@@ -104,6 +109,7 @@ __global__ void __launch_bounds__(FTHREADS) fp32_attn_kernel(const F32Params p) 
   }
 
   for (int jb = jb_lo; jb < jb_hi; ++jb) {
+    if (jb >= gap_lo && jb < gap_hi) continue;
     const int k0 = jb * FBN;
     __syncthreads();
     for (int x = tid; x < FBN * E / 4; x += FTHREADS) {
@@ -158,7 +164,7 @@ __global__ void __launch_bounds__(FTHREADS) fp32_attn_kernel(const F32Params p) 
       for (int c = 0; c < 8; ++c) {
         const int key = k0 + cg + 8 * c;
         float zz = RBF ? (2.f * p.scale) * z[r][c] - p.scale * sm.kn[cg + 8 * c] : p.scale * z[r][c];
-        if (key < lo_i[r] || key >= hi_i[r]) zz = -INFINITY;
+        if (key >= hi_i[r] || (key < lo_i[r] && key >= p.keep)) zz = -INFINITY;
         if (p.bias != nullptr && i < p.L && key < p.S) zz += p.bias[(size_t)i * p.S + key];
         z[r][c] = zz;
         mt = fmaxf(mt, zz);
@@ -240,6 +246,7 @@ int launch_f32_impl(const AttnArgs& a, cudaStream_t stream) {
   p.group = a.Hq / a.H;
   p.mask_kind = a.mask_kind;
   p.window = a.window;
+  p.keep = a.keep;
   p.scale = a.scale;
   const int smem = sizeof(F32Smem<E, EV>);
   auto kern = fp32_attn_kernel<E, EV, RBF>;

@@ -6,7 +6,9 @@
 
 namespace attn {
 
-enum MaskKind { MASK_NONE = 0, MASK_CAUSAL = 1, MASK_WINDOW = 2 };
+// MASK_STREAM: the sliding window plus the first `keep` keys, which stay visible
+// to every query at or after them (StreamingLLM's kept initial tokens).
+enum MaskKind { MASK_NONE = 0, MASK_CAUSAL = 1, MASK_WINDOW = 2, MASK_STREAM = 3 };
 
 // Validated arguments of one forward call (see include/attn_b200.h).
 struct AttnArgs {
@@ -22,6 +24,7 @@ struct AttnArgs {
   int mask_kind;
   int window;
   const float* bias;   // [L, S] or nullptr
+  int keep;            // MASK_STREAM: number of initial keys always visible (0 otherwise)
 };
 
 constexpr float LOG2E = 1.4426950408889634f;

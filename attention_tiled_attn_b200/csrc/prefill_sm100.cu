@@ -53,6 +53,7 @@ struct PrefillParams {
   int n_rb;         // ceil(L / BM)
   int n_items;
   int mask_kind, window;
+  int keep;         // streaming mask: initial keys visible to every later query
   float c_dot;      // scale * log2e           (dot)
   float c_rbf;      // 2 * scale * log2e       (rbf)
   float c_kn;       // scale * log2e           (rbf key-norm penalty)
@@ -118,16 +119,25 @@ struct TileInfo {
   int jb_lo, jb_hi;  // key-tile range [jb_lo, jb_hi)
 };
 
-__device__ __forceinline__ void tile_range(const PrefillParams& p, TileInfo& t) {
+// Key-tile range of a query tile; with the streaming mask also the first tile
+// past the kept initial keys (*gap_lo) and the first tile of the window of the
+// tile's first row (*gap_hi): the tiles in between no row of the tile sees.
+__device__ __forceinline__ void tile_range(const PrefillParams& p, TileInfo& t, int* gap_lo, int* gap_hi) {
   t.jb_lo = t.jb_hi = 0;
+  *gap_lo = *gap_hi = -1;
   if (!t.active) return;
   const int off = p.S - p.L;
   const int r_last = min(t.r0 + BM - 1, p.L - 1);
   const int hi = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, r_last + off + 1);
-  const int lo = (p.mask_kind == MASK_WINDOW) ? max(0, t.r0 + off - p.window + 1) : 0;
+  const int win_lo = max(0, t.r0 + off - p.window + 1);  // the first row's window start
+  const int lo = (p.mask_kind == MASK_WINDOW || (p.mask_kind == MASK_STREAM && p.keep == 0)) ? win_lo : 0;
   if (hi <= lo) return;
   t.jb_lo = lo / BN;
   t.jb_hi = (hi + BN - 1) / BN;
+  if (p.mask_kind == MASK_STREAM && p.keep > 0 && (p.keep + BN - 1) / BN < win_lo / BN) {
+    *gap_lo = (p.keep + BN - 1) / BN;
+    *gap_hi = win_lo / BN;
+  }
 }
 
 __device__ __forceinline__ bool in_range(const TileInfo& t, int jb) { return jb >= t.jb_lo && jb < t.jb_hi; }
@@ -152,7 +162,17 @@ struct Item {
   int n, kvh;
   TileInfo tile[2];
   int u_lo, u_hi;
+  int g_lo, g_hi;  // key tiles [g_lo, g_hi) of the union range are skipped (-1: none)
 };
+
+// Next key tile of an item after jb.  With the streaming mask every role steps
+// over the gap, so those tiles are never loaded and take no ring slot.  Without
+// it (STREAM false) this is jb + 1 and the gap fields are never read.
+template <bool STREAM>
+__device__ __forceinline__ int next_jb(const Item& w, int jb) {
+  if constexpr (STREAM) return (jb + 1 == w.g_lo) ? w.g_hi : jb + 1;
+  return jb + 1;
+}
 
 __device__ __forceinline__ void decode_item(const PrefillParams& p, int item, Item& w) {
   if (p.head_pairs) {
@@ -177,12 +197,23 @@ __device__ __forceinline__ void decode_item(const PrefillParams& p, int item, It
     w.tile[0] = {1, hq, 2 * rp * BM, 0, 0};
     w.tile[1] = {(2 * rp + 1) * BM < p.L ? 1 : 0, hq, (2 * rp + 1) * BM, 0, 0};
   }
-  tile_range(p, w.tile[0]);
-  tile_range(p, w.tile[1]);
+  int gl0, gh0, gl1, gh1;
+  tile_range(p, w.tile[0], &gl0, &gh0);
+  tile_range(p, w.tile[1], &gl1, &gh1);
   const bool h0 = w.tile[0].jb_hi > w.tile[0].jb_lo;
   const bool h1 = w.tile[1].jb_hi > w.tile[1].jb_lo;
   w.u_lo = w.u_hi = 0;
+  w.g_lo = h0 ? gl0 : gl1;
+  w.g_hi = h0 ? gh0 : gh1;
   if (h0 && h1) {
+    // Both tiles skip only the gap they share (the earlier row block's; the gaps
+    // start at the same tile).  The issuer frees a V slot once every tile that
+    // reads it has issued its PV; that needs the two tiles' key-tile lists to nest
+    // as with the causal mask.  A later row block's wider gap would let its pending
+    // PV fall behind the other tile's and hold the slot.  The one or two extra key
+    // tiles the later block reads are masked out whole.
+    w.g_hi = (gh0 < 0 || gh1 < 0) ? -1 : min(gh0, gh1);
+    if (w.g_hi < 0) w.g_lo = -1;
     w.u_lo = min(w.tile[0].jb_lo, w.tile[1].jb_lo);
     w.u_hi = max(w.tile[0].jb_hi, w.tile[1].jb_hi);
   } else if (h0) {
@@ -198,7 +229,9 @@ __device__ __forceinline__ void decode_item(const PrefillParams& p, int item, It
 // (k even) or k*G + G-1-b (k odd), so the heavy items spread evenly.
 __device__ __forceinline__ int snake_item(int b, int k, int G) { return k * G + ((k & 1) ? (G - 1 - b) : b); }
 
-template <int E, int EV, bool RBF>
+// STREAM: the streaming mask with kept initial keys (a compile-time switch, so the
+// other masks carry none of its bookkeeping in the softmax warps' registers).
+template <int E, int EV, bool RBF, bool STREAM>
 __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
@@ -269,7 +302,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
         if (w.u_hi <= w.u_lo) continue;
         const bool h0 = w.tile[0].jb_hi > w.tile[0].jb_lo, h1 = w.tile[1].jb_hi > w.tile[1].jb_lo;
         bool q_pending = true;
-        for (int jb = w.u_lo; jb < w.u_hi; ++jb, ++gk) {
+        for (int jb = w.u_lo; jb < w.u_hi; jb = next_jb<STREAM>(w, jb), ++gk) {
           const uint32_t ks = gk % C::NK, vs = gk % C::NV;
           if (!wait_bar(bar(C::B_KEMPTY + ks), ((gk / C::NK) & 1) ^ 1, abort_flag)) {
             ok = false;
@@ -330,12 +363,14 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
         ++qc;
         tc_fence_after();
         const uint32_t gbase = gk;
-        int pend0 = -1, pend1 = -1;
+        int pend0 = -1, pend1 = -1;  // key tile whose PV is still to issue, per query tile
         bool first0 = true, first1 = true;
         int v_waited = w.u_lo - 1, v_cur = -1, v_cur_uses = 0;
 
         auto issue_pv = [&](int t, int jbp) -> bool {
-          const uint32_t gp = gbase + (jbp - w.u_lo);
+          // ring position of key tile jbp: tiles past the gap sit g_hi - g_lo places earlier
+          uint32_t gp = gbase + (jbp - w.u_lo);
+          if constexpr (STREAM) gp -= (w.g_lo >= 0 && jbp >= w.g_hi) ? (w.g_hi - w.g_lo) : 0;
           const uint32_t vs = gp % C::NV;
           if (jbp > v_waited) {
             if (!wait_bar(bar(C::B_VFULL + vs), (gp / C::NV) & 1, abort_flag)) return false;
@@ -384,7 +419,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
           mma_commit(bar(C::B_SFULL + t));
         };
 
-        for (int jb = w.u_lo; ok && jb < w.u_hi; ++jb, ++gk) {
+        for (int jb = w.u_lo; ok && jb < w.u_hi; jb = next_jb<STREAM>(w, jb), ++gk) {
           const uint32_t ks = gk % C::NK;
           if (!wait_bar(bar(C::B_KFULL + ks), (gk / C::NK) & 1, abort_flag)) {
             ok = false;
@@ -402,13 +437,6 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
             pend1 = jb;
           }
           mma_commit(bar(C::B_KEMPTY + ks));
-          if (!in_range(w.tile[0], jb) && !in_range(w.tile[1], jb)) {
-            // a key tile neither query tile reads: let its V copy land, then free the slot
-            const uint32_t vs = gk % C::NV;
-            if (!wait_bar(bar(C::B_VFULL + vs), (gk / C::NV) & 1, abort_flag)) { ok = false; break; }
-            mma_commit(bar(C::B_VEMPTY + vs));
-            if (jb > v_waited) v_waited = jb;
-          }
         }
         if (!ok) break;
         mma_commit(bar(C::B_QEMPTY));  // all QK^T of this item issued: Q may be replaced
@@ -437,7 +465,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
       if (item >= p.n_items) continue;
       Item w;
       decode_item(p, item, w);
-      for (int jb = w.u_lo; jb < w.u_hi; ++jb, ++gk) {
+      for (int jb = w.u_lo; jb < w.u_hi; jb = next_jb<STREAM>(w, jb), ++gk) {
         const uint32_t ks = gk % C::NK;
         const uint32_t slot = gk % C::NKN;
         const bool w1 = wait_bar(bar(C::B_KFULL + ks), (gk / C::NK) & 1, abort_flag);
@@ -496,7 +524,8 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
       decode_item(p, item, w);
       const TileInfo T = t ? w.tile[1] : w.tile[0];
       const int i = T.r0 + row;
-      const int lo_i = (p.mask_kind == MASK_WINDOW) ? (i + off - p.window + 1) : 0;
+      // key j visible to row i iff lo_i <= j < hi_i (streaming mask: or j < keep)
+      const int lo_i = (STREAM || p.mask_kind == MASK_WINDOW) ? (i + off - p.window + 1) : 0;
       const int hi_i = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, i + off + 1);
       const int first_row_hi = T.r0 + off + 1;  // key limit of the tile's first row
       const int last_row_lo = min(T.r0 + BM - 1, p.L - 1) + off - p.window + 1;
@@ -504,7 +533,11 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
 
       float m_run = -INFINITY, l_run = 0.f;
       int it = 0;
-      for (int jb = w.u_lo; jb < w.u_hi; ++jb, ++gk) {
+      // RBF: walk the item's union range, which the key-norm ring follows; dot: only
+      // this tile's own key tiles (fewer live values in the softmax warps)
+      const int j_lo = RBF ? w.u_lo : T.jb_lo;
+      const int j_hi = RBF ? w.u_hi : T.jb_hi;
+      for (int jb = j_lo; jb < j_hi; jb = next_jb<STREAM>(w, jb), ++gk) {
         const uint32_t slot = gk % C::NKN;
         if (RBF) {
           const bool wk = wait_bar(bar(C::B_KNFULL + slot), (gk / C::NKN) & 1, abort_flag);
@@ -512,10 +545,10 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
             ok = false;
             break;
           }
-        }
-        if (!in_range(T, jb)) {
-          if (RBF) mbar_arrive(bar(C::B_KNEMPTY + slot));
-          continue;
+          if (!in_range(T, jb)) {
+            mbar_arrive(bar(C::B_KNEMPTY + slot));
+            continue;
+          }
         }
         {
           const bool ws = wait_bar(bar(C::B_SFULL + t), sc & 1, abort_flag);
@@ -544,7 +577,8 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
 
         const int k0 = jb * BN;
         const bool need_mask = ((k0 + BN) > p.S) || (p.mask_kind != MASK_NONE && (k0 + BN) > first_row_hi) ||
-                               (p.mask_kind == MASK_WINDOW && k0 < last_row_lo);
+                               ((STREAM || p.mask_kind == MASK_WINDOW) && k0 < last_row_lo &&
+                                (!STREAM || k0 + BN > p.keep));
         // Logits stay in "exponent units" u with  base-2 logit = u * c_exp:
         //   dot: u = q.k (+ bias / scale),  c_exp = scale * log2e
         //   rbf: u = 2*scale*log2e*q.k - scale*log2e*||k||^2 (+ bias * log2e),  c_exp = 1
@@ -562,9 +596,21 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
         }
         if (need_mask) {
           const int lo = lo_i - k0, hi = hi_i - k0;
+          if constexpr (STREAM) {
+            // two passes, so no more than two bounds are live at once: keys past the
+            // row's causal limit, then those between the kept keys and the window
 #pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c < lo || c >= hi) z[c] = -INFINITY;
+            for (int c = 0; c < BN; ++c)
+              if (c >= hi) z[c] = -INFINITY;
+            const int kp = p.keep - k0;
+#pragma unroll
+            for (int c = 0; c < BN; ++c)
+              if (c >= kp && c < lo) z[c] = -INFINITY;
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN; ++c)
+              if (c < lo || c >= hi) z[c] = -INFINITY;
+          }
         }
         if (has_bias && bias_row != nullptr) {
           const int lim = p.S - k0;
@@ -702,7 +748,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-template <int E, int EV, bool RBF>
+template <int E, int EV, bool RBF, bool STREAM>
 int launch_impl(const AttnArgs& a, cudaStream_t stream) {
   using C = Cfg<E, EV, RBF>;
   CUtensorMap tq, tk, tv;
@@ -726,14 +772,16 @@ int launch_impl(const AttnArgs& a, cudaStream_t stream) {
     p.n_items = p.N * p.H * (p.group / 2) * p.n_rb;
   else
     p.n_items = p.N * p.Hq * ((p.n_rb + 1) / 2);
-  p.mask_kind = a.mask_kind;
+  // the streaming mask without kept keys is the sliding window
+  p.mask_kind = (a.mask_kind == MASK_STREAM && !STREAM) ? MASK_WINDOW : a.mask_kind;
   p.window = a.window;
+  p.keep = STREAM ? a.keep : 0;
   p.c_dot = a.scale * LOG2E;
   p.c_rbf = 2.f * a.scale * LOG2E;
   p.c_kn = a.scale * LOG2E;
   p.c_exp = RBF ? 1.f : a.scale * LOG2E;
   p.c_bias = RBF ? LOG2E : 1.f / a.scale;
-  auto kern = prefill_kernel<E, EV, RBF>;
+  auto kern = prefill_kernel<E, EV, RBF, STREAM>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return -13;
   {
@@ -771,9 +819,12 @@ unsigned int take_status_prefill(cudaStream_t s) { return take_device_status_loc
 
 int launch_prefill_bf16(const AttnArgs& a, cudaStream_t stream) {
   const bool r = a.rbf;
-#define ATTN_PREFILL_CASE(e, ev)                                            \
-  if (a.E == e && a.Ev == ev) return r ? launch_impl<e, ev, true>(a, stream) \
-                                       : launch_impl<e, ev, false>(a, stream);
+  const bool st = a.mask_kind == MASK_STREAM && a.keep > 0;
+#define ATTN_PREFILL_CASE(e, ev)                                                                 \
+  if (a.E == e && a.Ev == ev) {                                                                  \
+    if (st) return r ? launch_impl<e, ev, true, true>(a, stream) : launch_impl<e, ev, false, true>(a, stream); \
+    return r ? launch_impl<e, ev, true, false>(a, stream) : launch_impl<e, ev, false, false>(a, stream); \
+  }
   ATTN_PREFILL_CASE(64, 64)
   ATTN_PREFILL_CASE(128, 128)
   ATTN_PREFILL_CASE(64, 128)

@@ -60,31 +60,47 @@ NCU_TRAFFIC_BYTES = {
 # algorithmic work
 # ---------------------------------------------------------------------------
 
+def row_pairs(r: sw.Recipe, rows) -> np.ndarray:
+    """Visible keys of each query row in ``rows`` under r's mask kind (a bias does not change it)."""
+    ip = np.asarray(rows, dtype=np.int64) + (r.S - r.L)
+    if r.mask_kind == "none":
+        return np.full(ip.size, r.S, dtype=np.int64)
+    hi = np.minimum(r.S, ip + 1)
+    if r.mask_kind == "causal":
+        return np.maximum(0, hi)
+    lo = np.minimum(np.maximum(0, ip - r.window + 1), np.maximum(hi, 0))
+    n = np.maximum(0, hi - lo)
+    if r.mask_kind == "streaming":
+        n = n + np.maximum(0, np.minimum(r.keep, lo))  # kept initial keys below the window
+    return n
+
+
 def visible_pairs(r: sw.Recipe) -> int:
     """Number of (query, key) pairs the mask leaves visible, per (n, hq)."""
-    i = np.arange(r.L, dtype=np.int64)
-    ip = i + (r.S - r.L)
-    if r.mask_kind == "none" or r.bias != "none":
-        hi = np.full(r.L, r.S, dtype=np.int64)
-        lo = np.zeros(r.L, dtype=np.int64)
-        if r.mask_kind != "none":
-            hi = np.minimum(r.S, ip + 1)
-            if r.mask_kind == "window":
-                lo = np.maximum(0, ip - r.window + 1)
-    else:
-        hi = np.minimum(r.S, ip + 1)
-        lo = np.maximum(0, ip - r.window + 1) if r.mask_kind == "window" else np.zeros(r.L, dtype=np.int64)
-    return int(np.maximum(0, hi - lo).sum())
+    return int(row_pairs(r, np.arange(r.L)).sum())
 
 
 def is_decode(r: sw.Recipe) -> bool:
     return r.dtype == "bf16" and r.mode == "dot" and (r.Hq // r.H) * r.L <= 16
 
 
+def decode_keys(r: sw.Recipe) -> int:
+    """Keys some query row can see: what a decode step has to read from the cache."""
+    if r.mask_kind in ("none", "causal"):
+        return r.S
+    ip = np.arange(r.L, dtype=np.int64)[:, None] + (r.S - r.L)
+    j = np.arange(r.S, dtype=np.int64)[None, :]
+    d = ip - j
+    seen = (d >= 0) & (d < r.window)
+    if r.mask_kind == "streaming":
+        seen |= (d >= 0) & (j < r.keep)
+    return int(seen.any(axis=0).sum())
+
+
 def work_units(r: sw.Recipe):
     """(amount, unit, roofline bound) of one step of workload r on one GPU."""
     if is_decode(r):
-        kv_bytes = r.N * r.H * r.S * (r.E + r.Ev) * 2
+        kv_bytes = r.N * r.H * decode_keys(r) * (r.E + r.Ev) * 2
         return kv_bytes, "GB/s", "hbm"
     flops = 2 * (r.E + r.Ev) * visible_pairs(r) * r.N * r.Hq
     return flops, "TFLOP/s", "tensor"
@@ -233,7 +249,7 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
 
     def step():
         attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=r.mode, sink=t["sink"], mask_kind=r.mask_kind,
-                      window=r.window, bias=t["bias"], out=out, lse=lse, stream=stream)
+                      window=r.window, keep_first=r.keep, bias=t["bias"], out=out, lse=lse, stream=stream)
 
     amount, unit, bound = work_units(r)
     barrier(pg)
@@ -292,8 +308,8 @@ def e2e_measure(res, steps, warmup):
         for k in ("q", "k", "v"):
             dev[k].copy_(host[k], non_blocking=True)
         attn.attn_fwd(dev["q"], dev["k"], dev["v"], scale=r.scale, mode=r.mode, sink=t["sink"],
-                      mask_kind=r.mask_kind, window=r.window, bias=t["bias"], out=res["out"], lse=res["lse"],
-                      stream=stream)
+                      mask_kind=r.mask_kind, window=r.window, keep_first=r.keep, bias=t["bias"], out=res["out"],
+                      lse=res["lse"], stream=stream)
         out_host.copy_(res["out"], non_blocking=True)
         lse_host.copy_(res["lse"], non_blocking=True)
 
@@ -341,19 +357,14 @@ class OracleSample:
 
     def rows_amount(self, rows):
         r = self.r
-        ip = rows + (r.S - r.L)
-        hi = np.full(rows.size, r.S) if r.mask_kind == "none" or r.bias != "none" else np.minimum(r.S, ip + 1)
-        if r.mask_kind != "none" and r.bias != "none":
-            hi = np.minimum(r.S, ip + 1)
-        lo = np.maximum(0, ip - r.window + 1) if r.mask_kind == "window" else np.zeros(rows.size)
-        return float(np.maximum(0, hi - lo).sum()) * self.per_pair
+        return float(row_pairs(r, rows).sum()) * self.per_pair
 
     def run(self, rows):
         r = self.r
         for i0 in range(0, rows.size, 256):
             rr = rows[i0:i0 + 256]
             self.orc.attend_rows(self.q[rr], rr, self.k, self.v, r.L, scale=r.scale, mode=r.mode, sink=self.sink,
-                                 mask_kind=r.mask_kind, window=r.window,
+                                 mask_kind=r.mask_kind, window=r.window, keep=r.keep,
                                  bias_rows=None if self.bias is None else self.bias[rr])
         return self.rows_amount(rows)
 
@@ -418,6 +429,12 @@ def ours(args):
                 runs.append((name + ":dot_control", dataclasses.replace(r0, mode="dot")))
             if r0.sink != "none":
                 runs.append((name + ":no_sink_control", dataclasses.replace(r0, sink="none")))
+            # StreamingLLM variant: 4 kept initial tokens plus the window (decode: a 4096-key window)
+            if r0.mask_kind == "window":
+                runs.append((name + ":streaming_keep4", dataclasses.replace(r0, mask_kind="streaming", keep=4)))
+            elif is_decode(r0):
+                runs.append((name + ":streaming_keep4_w4096",
+                             dataclasses.replace(r0, mask_kind="streaming", window=4096, keep=4)))
         for label, rr in runs:
             base = sw.RECIPES[rr.name]
             sw.RECIPES[rr.name] = rr

@@ -66,7 +66,8 @@ typedef enum {
   ATTN_ERR_DEVICE_TIMEOUT = -14,/* a kernel gave up a bounded wait (see attn_device_status) */
   ATTN_ERR_DEVICE = -15,        /* the current device is not sm_100 */
   ATTN_ERR_SCRATCH_LIMIT = -16, /* attn_decode_fwd_noalloc: the call needs more scratch than the fixed area holds */
-  ATTN_ERR_NOT_DECODE = -17     /* attn_decode_fwd_noalloc: not a decode-shaped bf16 call ((Hq/H)*L <= 16, dot) */
+  ATTN_ERR_NOT_DECODE = -17,    /* attn_decode_fwd_noalloc: not a decode-shaped bf16 call ((Hq/H)*L <= 16, dot) */
+  ATTN_ERR_KEEP = -18           /* attn_fwd_streaming: keep_first < 0 */
 } attn_status;
 
 /*
@@ -104,6 +105,26 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
              int N, int Hq, int H, int L, int S, int E, int Ev, float scale, int mode,
              const float* sink_logits, int mask_kind, int window, const float* bias,
              int dtype, void* stream);
+
+/*
+ * attn_fwd_streaming -- attn_fwd under the StreamingLLM visibility rule: the
+ * first keep_first keys (the attention-sink tokens) stay visible to every later
+ * query, and otherwise only the last `window` keys are (page "Attention Sink"
+ * section 3.2: keep the initial tokens' KV plus a rolling window of recent
+ * ones).  With i' = i + (S - L):
+ *   key j visible iff  j <= i'  and  (j < keep_first  or  i' - j < window)
+ * keep_first = 0 is the sliding window; keep_first >= S is the causal mask.
+ *
+ * Every other argument, layout, ownership rule, dispatch and status code is
+ * attn_fwd's (the mask_kind argument is replaced by window and keep_first).
+ * Returns ATTN_ERR_WINDOW for window < 1 and ATTN_ERR_KEEP for keep_first < 0.
+ * The kernels read only the key tiles some query of a tile can see: the keys
+ * between the kept ones and the window are never loaded.
+ */
+int attn_fwd_streaming(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int N, int Hq, int H, int L, int S, int E, int Ev, float scale, int mode,
+                       const float* sink_logits, int window, int keep_first, const float* bias,
+                       int dtype, void* stream);
 
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* attn_status_string(int status);

@@ -23,6 +23,9 @@ in blocks of query rows so that memory stays bounded:
     causal  key j visible iff j <= i'
     window  key j visible iff 0 <= i' - j < W   (W keys, self included)
   and an additive bias B[i, j] (0 or -inf) composes with either.
+* StreamingLLM mask (page "Attention Sink" §3.2: keep the first tokens'
+  KV plus a rolling window of recent tokens): with R kept initial tokens,
+    streaming  key j visible iff j <= i'  and  (j < R  or  i' - j < W)
 * Grouped-query attention (page "SDPA란 무엇인가" §5): query head hq reads
   KV head hq // (Hq // H).
 * Sink (page "Attention Sink" §4.2, §5.2-5.4): a per-query-head logit s_h
@@ -40,10 +43,11 @@ import numpy as np
 NEG_INF = -np.inf
 
 
-def visible(rows: np.ndarray, S: int, L: int, mask_kind: str, window: int = 0) -> np.ndarray:
+def visible(rows: np.ndarray, S: int, L: int, mask_kind: str, window: int = 0, keep: int = 0) -> np.ndarray:
     """Boolean (R, S) visibility of keys 0..S-1 for query positions ``rows``.
 
     Bottom-right alignment: query i sits at key position i' = i + (S - L).
+    ``keep`` is the number of initial tokens the streaming mask keeps.
     """
     rows = np.asarray(rows, dtype=np.int64)
     ip = rows[:, None] + (S - L)
@@ -57,6 +61,11 @@ def visible(rows: np.ndarray, S: int, L: int, mask_kind: str, window: int = 0) -
             raise ValueError("window must be >= 1")
         d = ip - j
         return (d >= 0) & (d < window)
+    if mask_kind == "streaming":
+        if window < 1 or keep < 0:
+            raise ValueError("streaming mask needs window >= 1 and keep >= 0")
+        d = ip - j
+        return (d >= 0) & ((j < keep) | (d < window))
     raise ValueError(f"unknown mask kind {mask_kind!r}")
 
 
@@ -100,7 +109,7 @@ def softmax_with_sink(z: np.ndarray, vis: np.ndarray, sink: float | None):
 
 
 def attend_rows(q_rows, rows, k, v, L, *, scale, mode="dot", sink=None, mask_kind="none",
-                window=0, bias_rows=None, return_weights=False):
+                window=0, bias_rows=None, return_weights=False, keep=0):
     """Attention of query rows ``q_rows`` (R, E) at positions ``rows`` against one KV head.
 
     k (S, E), v (S, Ev), bias_rows (R, S) or None.  Returns out (R, Ev) and
@@ -112,7 +121,7 @@ def attend_rows(q_rows, rows, k, v, L, *, scale, mode="dot", sink=None, mask_kin
     z = logits(q_rows, k, scale, mode)
     if bias_rows is not None:
         z = z + np.asarray(bias_rows, dtype=np.float64)
-    vis = visible(rows, S, L, mask_kind, window)
+    vis = visible(rows, S, L, mask_kind, window, keep)
     alpha, p_sink, lse = softmax_with_sink(z, vis, sink)
     out = alpha @ v
     if return_weights:
@@ -121,7 +130,7 @@ def attend_rows(q_rows, rows, k, v, L, *, scale, mode="dot", sink=None, mask_kin
 
 
 def attention_forward(q, k, v, *, scale, mode="dot", sink=None, mask_kind="none", window=0,
-                      bias=None, row_block=128):
+                      bias=None, row_block=128, keep=0):
     """Whole forward: q (N,Hq,L,E), k (N,H,S,E), v (N,H,S,Ev) float64.
 
     sink: per-query-head logits (Hq,) or None.  bias: (L, S) or None.
@@ -145,7 +154,7 @@ def attention_forward(q, k, v, *, scale, mode="dot", sink=None, mask_kind="none"
                 b = None if bias is None else np.asarray(bias)[rows]
                 o, l = attend_rows(q[n, hq, rows], rows, k[n, kvh], v[n, kvh], L, scale=scale,
                                    mode=mode, sink=s, mask_kind=mask_kind, window=window,
-                                   bias_rows=b)
+                                   bias_rows=b, keep=keep)
                 out[n, hq, rows] = o
                 lse[n, hq, rows] = l
     return out, lse

@@ -222,8 +222,9 @@ class Recipe:
     dtype: str            # "bf16" or "f32"
     mode: str             # "dot" or "rbf"
     scale: float
-    mask_kind: str        # "none", "causal", "window"
+    mask_kind: str        # "none", "causal", "window", "streaming"
     window: int = 0
+    keep: int = 0         # streaming mask: initial tokens every later query sees
     sink: str = "none"    # "none", "fixed", "normal"
     sink_values: tuple = ()
     bias: str = "none"    # "none" or "random10"

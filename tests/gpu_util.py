@@ -20,16 +20,13 @@ BF16_ABS = 2e-2
 BF16_REL_L2 = 5e-3
 BF16_LSE = 1e-3
 
-MASK_NAME = {"none": "none", "causal": "causal", "window": "window"}
-
-
 def api_mode(r: sw.Recipe) -> str:
     return r.mode  # "dot" or "rbf"; a sink applies whenever sink logits are passed
 
 
 def run_gpu(r: sw.Recipe, t: dict):
     out, lse = attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=api_mode(r), sink=t["sink"],
-                             mask_kind=r.mask_kind, window=r.window, bias=t["bias"])
+                             mask_kind=r.mask_kind, window=r.window, bias=t["bias"], keep_first=r.keep)
     torch.cuda.synchronize()
     return out, lse
 
@@ -55,7 +52,7 @@ def oracle_rows(r: sw.Recipe, n: int, hq: int, rows, host: dict | None = None):
     s = None if sink is None else float(sink[hq])
     b = None if bias is None else bias[rows].astype(np.float64)
     return orc.attend_rows(q[rows], rows, k, v, r.L, scale=r.scale, mode=r.mode, sink=s,
-                           mask_kind=r.mask_kind, window=r.window, bias_rows=b)
+                           mask_kind=r.mask_kind, window=r.window, bias_rows=b, keep=r.keep)
 
 
 def compare(r: sw.Recipe, got_out, got_lse, ref_out, ref_lse, what=""):
@@ -99,7 +96,7 @@ def run_and_check_full(r: sw.Recipe):
     ref_out, ref_lse = orc.attention_forward(
         sw.as_f64(r, host["q"]), sw.as_f64(r, host["k"]), sw.as_f64(r, host["v"]), scale=r.scale, mode=r.mode,
         sink=None if host["sink"] is None else host["sink"].astype(np.float64), mask_kind=r.mask_kind,
-        window=r.window, bias=None if host["bias"] is None else host["bias"].astype(np.float64))
+        window=r.window, bias=None if host["bias"] is None else host["bias"].astype(np.float64), keep=r.keep)
     return compare(r, out_to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, r.name)
 
 

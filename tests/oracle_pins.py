@@ -346,10 +346,39 @@ def check_gqa_repeat(seed=13):
         assert np.array_equal(a, b) and np.array_equal(la, lb)
 
 
+def check_streaming_mask(seed=14):
+    """StreamingLLM mask: keep = 0 is the sliding window, keep >= i'+1 is causal,
+    the visible count is |{j < keep} u {i'-W < j <= i'}|, and a decode query over
+    the whole cache equals plain attention over the compacted cache (the kept
+    first tokens followed by the last W tokens)."""
+    rng = np.random.default_rng(seed)
+    L, S = 6, 20
+    for W, keep in ((3, 0), (4, 2), (5, 7), (20, 1)):
+        vis = orc.visible(np.arange(L), S, L, "streaming", W, keep)
+        if keep == 0:
+            assert np.array_equal(vis, orc.visible(np.arange(L), S, L, "window", W))
+        for i in range(L):
+            ip = i + S - L
+            want = {j for j in range(S) if j <= ip and (j < keep or ip - j < W)}
+            assert set(np.nonzero(vis[i])[0].tolist()) == want
+    assert np.array_equal(orc.visible(np.arange(L), S, L, "streaming", 2, S),
+                          orc.visible(np.arange(L), S, L, "causal"))
+    for mode in ("dot", "rbf"):
+        for W, keep in ((5, 3), (1, 4), (7, 0)):
+            q = _rand(rng, 1, 2, 1, 4)
+            k, v = _rand(rng, 1, 1, S, 4), _rand(rng, 1, 1, S, 3)
+            sink = np.array([0.3, -0.7])
+            full, lf = orc.attention_forward(q, k, v, scale=0.6, mode=mode, sink=sink, mask_kind="streaming",
+                                             window=W, keep=keep)
+            idx = list(range(keep)) + list(range(S - W, S))
+            comp, lc = orc.attention_forward(q, k[:, :, idx], v[:, :, idx], scale=0.6, mode=mode, sink=sink)
+            assert np.allclose(full, comp, atol=1e-13) and np.allclose(lf, lc, atol=1e-13), (mode, W, keep)
+
+
 ALL_CHECKS = [
     check_dot_matches_sdpa, check_brute_force, check_rbf_expansion, check_rbf_limits,
     check_dot_limits, check_uniform_entropy_golden, check_sink_limit, check_sink_mass,
     check_zero_sink_equivalence, check_convexity, check_causal_alignment_golden,
     check_fully_masked_rows, check_window_semantics, check_permutation_equivariance,
-    check_gqa_repeat,
+    check_gqa_repeat, check_streaming_mask,
 ]

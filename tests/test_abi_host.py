@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_status_strings(lib):
     assert attn.status_string(0) == "ok"
-    for st in range(-15, 0):
+    for st in range(-18, 0):
         s = attn.status_string(st)
         assert s and s != "unknown status"
     assert attn.status_string(-99) == "unknown status"
@@ -74,6 +74,24 @@ def call(**kw):
 ])
 def test_argument_validation(lib, kw, status):
     assert call(**kw) == status
+
+
+def call_streaming(**kw):
+    a = dict(q=P, k=P, v=P, out=P, lse=P, N=1, Hq=2, H=1, L=8, S=8, E=64, Ev=64, scale=0.125, mode=0,
+             sink=None, window=4, keep=2, bias=None, dtype=0, stream=None)
+    a.update(kw)
+    return attn.attn_fwd_streaming_raw(a["q"], a["k"], a["v"], a["out"], a["lse"], a["N"], a["Hq"], a["H"], a["L"],
+                                       a["S"], a["E"], a["Ev"], a["scale"], a["mode"], a["sink"], a["window"],
+                                       a["keep"], a["bias"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(window=0), -8), (dict(window=-5), -8), (dict(keep=-1), -18),
+    (dict(q=None), -1), (dict(Hq=3, H=2), -3), (dict(E=96), -4), (dict(scale=0.0), -5),
+    (dict(mode=2, sink=None), -9), (dict(dtype=2), -10), (dict(k=P + 8), -11),
+])
+def test_streaming_argument_validation(lib, kw, status):
+    assert call_streaming(**kw) == status
 
 
 def test_python_binding_rejects_cpu_tensors(lib):

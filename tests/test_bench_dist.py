@@ -66,3 +66,23 @@ def test_visible_pairs_closed_forms():
     assert bench.visible_pairs(r2) == 2048 * 2048
     amount, unit, bound = bench.work_units(sw.RECIPES["decode_sink_gqa_128k_bf16"])
     assert (amount, unit, bound) == (32 * 8 * 131072 * 256 * 2, "GB/s", "hbm")
+
+
+def test_visible_pairs_and_decode_keys_match_the_oracle_mask():
+    """Work accounting of every mask kind against the oracle's visibility, by brute force."""
+    import dataclasses
+
+    import numpy as np
+
+    from oracle import attention as orc
+    from synth import workloads as sw
+    base = sw.RECIPES["tiny_rbf_sink_causal_f32"]
+    cases = [("none", 0, 0), ("causal", 0, 0), ("window", 7, 0), ("streaming", 7, 3), ("streaming", 5, 0),
+             ("streaming", 4, 200), ("streaming", 1, 1)]
+    for L, S in ((37, 37), (5, 60), (60, 20), (1, 90)):
+        for mk, w, keep in cases:
+            r = dataclasses.replace(base, L=L, S=S, mask_kind=mk, window=w, keep=keep)
+            vis = orc.visible(np.arange(L), S, L, mk, w, keep)
+            assert bench.visible_pairs(r) == int(vis.sum()), (L, S, mk, w, keep)
+            if mk in ("window", "streaming"):
+                assert bench.decode_keys(r) == int(vis.any(axis=0).sum()), (L, S, mk, w, keep)

@@ -32,16 +32,22 @@ def _dot_scale_dropped(q_rows, k, scale, mode, key_block=512):
     return _real_logits(q_rows, k, scale, mode, key_block)
 
 
-def _top_left(rows, S, L, mask_kind, window=0):
-    return _real_visible(rows, S, S, mask_kind, window)
+def _top_left(rows, S, L, mask_kind, window=0, keep=0):
+    return _real_visible(rows, S, S, mask_kind, window, keep)
 
 
-def _window_off_by_one(rows, S, L, mask_kind, window=0):
-    if mask_kind == "window":
+def _window_off_by_one(rows, S, L, mask_kind, window=0, keep=0):
+    if mask_kind in ("window", "streaming"):
         rows = np.asarray(rows)
         d = rows[:, None] + (S - L) - np.arange(S)[None, :]
-        return (d >= 0) & (d <= window)
-    return _real_visible(rows, S, L, mask_kind, window)
+        return (d >= 0) & ((d <= window) | (np.arange(S)[None, :] < keep))
+    return _real_visible(rows, S, L, mask_kind, window, keep)
+
+
+def _streaming_keep_ignored(rows, S, L, mask_kind, window=0, keep=0):
+    if mask_kind == "streaming":
+        return _real_visible(rows, S, L, "window", window)
+    return _real_visible(rows, S, L, mask_kind, window, keep)
 
 
 def _sink_in_values(z, vis, sink):
@@ -66,6 +72,8 @@ MUTATIONS = [
     ("visible", _top_left, pins.check_causal_alignment_golden),
     ("visible", _top_left, pins.check_dot_matches_sdpa),
     ("visible", _window_off_by_one, pins.check_window_semantics),
+    ("visible", _window_off_by_one, pins.check_streaming_mask),
+    ("visible", _streaming_keep_ignored, pins.check_streaming_mask),
     ("softmax_with_sink", _sink_in_values, pins.check_sink_mass),
     ("softmax_with_sink", _lse_without_sink, pins.check_brute_force),
 ]

@@ -49,6 +49,17 @@ PREFILL_CASES = [
     R("p_dot_window1_130", L=130, S=130, mask_kind="window", window=1),
     R("p_dot_none_600_g2_e128_sink", L=600, S=600, E=128, Ev=128, Hq=4, H=2, N=2, sink="normal",
       scale=0.0884),
+    # streaming mask: kept initial keys plus a window; key tiles in between are skipped
+    R("p_stream_keep4_w64_600_g2_sink", L=600, S=600, Hq=4, H=2, mask_kind="streaming", window=64, keep=4,
+      sink="normal"),
+    R("p_rbf_stream_keep130_w100_700_bias", L=700, S=700, E=128, Ev=128, mode="rbf", mask_kind="streaming",
+      window=100, keep=130, bias="random10", scale=0.05),
+    R("p_stream_keep0_w50_300", L=300, S=300, mask_kind="streaming", window=50, keep=0),
+    R("p_stream_keep_all_300", L=300, S=300, Hq=4, H=1, mask_kind="streaming", window=20, keep=1000),
+    R("p_stream_L200_S900_keep16_w128_e128", L=200, S=900, E=128, Ev=128, Hq=6, H=2, mask_kind="streaming",
+      window=128, keep=16, sink="normal", scale=0.0884),
+    R("p_stream_w1_keep1_520", L=520, S=520, mask_kind="streaming", window=1, keep=1),
+    R("p_stream_keep256_w128_1100", L=1100, S=1100, N=2, mask_kind="streaming", window=128, keep=256),
 ]
 
 FP32_CASES = [
@@ -59,6 +70,10 @@ FP32_CASES = [
     R("f_dot_causal_L1_S6", L=1, S=6, dtype="f32", mask_kind="causal"),
     R("f_dot_causal_L40_S10_empty", L=40, S=10, dtype="f32", mask_kind="causal", sink="fixed",
       sink_values=(0.5, -0.5)),
+    R("f_stream_keep5_w40_300_sink", L=300, S=300, Hq=4, H=2, dtype="f32", mask_kind="streaming", window=40,
+      keep=5, sink="normal"),
+    R("f_rbf_stream_keep70_w30_L100_S400", L=100, S=400, dtype="f32", mode="rbf", mask_kind="streaming",
+      window=30, keep=70, bias="random10"),
 ]
 
 DECODE_CASES = [
@@ -71,6 +86,14 @@ DECODE_CASES = [
     R("d_L3_g5_S129_e128_ev64", L=3, S=129, E=128, Ev=64, Hq=5, H=1),
     R("d_many_units", L=1, S=200, N=40, Hq=16, H=8, sink="normal"),
     R("d_L2_causal_S1_empty_row", L=2, S=1, Hq=2, H=2, mask_kind="causal"),
+    R("d_stream_L1_S5000_keep4_w1000_g4", L=1, S=5000, Hq=8, H=2, mask_kind="streaming", window=1000, keep=4,
+      sink="normal"),
+    R("d_stream_L3_S800_keep70_w100_g2_bias", L=3, S=800, Hq=4, H=2, mask_kind="streaming", window=100, keep=70,
+      bias="random10"),
+    R("d_stream_L1_S300_keep200_w150_overlap", L=1, S=300, mask_kind="streaming", window=150, keep=200),
+    R("d_stream_L2_S50_keep0_w10", L=2, S=50, mask_kind="streaming", window=10, keep=0),
+    R("d_stream_many_units", L=1, S=3000, N=40, Hq=16, H=8, E=128, Ev=128, mask_kind="streaming", window=256,
+      keep=4, scale=0.0884),
 ]
 
 

@@ -34,6 +34,13 @@ in blocks of query rows so that memory stays bounded:
   out = sum_{j in A} e^{z_j-M} v_j / D,  lse = M + ln D.
 * A row with no visible key and no sink gives out = 0 and lse = -inf (page
   "SDPA란 무엇인가" §4: SDPA returns 0 instead of NaN for a fully masked row).
+* Exact attention over a selected key subset (page "기술 요약: SOCKET - 희소
+  어텐션을 위한 SOft Collision Kernel EsTimator", 방법론, 핵심 메커니즘 step 4:
+  the top-k keys are picked, then exact attention runs on that subset): the
+  softmax and the value sum run over the listed keys of the KV head only, with
+  the mask taken at each key's original position.  One list per (batch, KV
+  head), shared by the group's query heads; entries outside [0, S) select
+  nothing; a repeated entry counts once per listing.
 """
 
 from __future__ import annotations
@@ -157,4 +164,47 @@ def attention_forward(q, k, v, *, scale, mode="dot", sink=None, mask_kind="none"
                                    bias_rows=b, keep=keep)
                 out[n, hq, rows] = o
                 lse[n, hq, rows] = l
+    return out, lse
+
+
+def select_keys(sel: np.ndarray, S: int) -> np.ndarray:
+    """The entries of a key list that name a cached key (0 <= j < S), in list order."""
+    sel = np.asarray(sel, dtype=np.int64)
+    return sel[(sel >= 0) & (sel < S)]
+
+
+def visible_at(rows, positions, S: int, L: int, mask_kind: str, window: int = 0) -> np.ndarray:
+    """Visibility (R, len(positions)) of keys at the given original positions."""
+    return visible(rows, S, L, mask_kind, window)[:, np.asarray(positions, dtype=np.int64)]
+
+
+def attention_over_index_set(q, k, v, key_idx, *, scale, sink=None, mask_kind="none", window=0, bias=None):
+    """Exact attention of every query row over the keys listed for its KV head.
+
+    q (N,Hq,L,E), k (N,H,S,E), v (N,H,S,Ev), key_idx (N,H,K) integer key
+    positions.  sink: (Hq,) or None; bias: (L, S) or None, read at the original
+    positions.  Returns out (N,Hq,L,Ev) and lse (N,Hq,L).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    N, Hq, L, _ = q.shape
+    H, S = k.shape[1], k.shape[2]
+    if Hq % H:
+        raise ValueError("Hq must be a multiple of H")
+    g = Hq // H
+    out = np.zeros((N, Hq, L, v.shape[3]), dtype=np.float64)
+    lse = np.zeros((N, Hq, L), dtype=np.float64)
+    rows = np.arange(L)
+    for n in range(N):
+        for hq in range(Hq):
+            kvh = hq // g
+            pos = select_keys(np.asarray(key_idx)[n, kvh], S)
+            z = logits(q[n, hq], k[n, kvh][pos], scale, "dot")
+            if bias is not None:
+                z = z + np.asarray(bias, dtype=np.float64)[:, pos]
+            vis = visible_at(rows, pos, S, L, mask_kind, window)
+            alpha, _, l = softmax_with_sink(z, vis, None if sink is None else float(sink[hq]))
+            out[n, hq] = alpha @ v[n, kvh][pos]
+            lse[n, hq] = l
     return out, lse

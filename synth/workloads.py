@@ -48,6 +48,7 @@ STREAM_V = 3
 STREAM_SINK = 4
 STREAM_BIAS = 5
 STREAM_KEY_FACTOR = 6
+STREAM_KEY_INDEX = 7
 
 LN2 = 0.6931471805599453          # double nearest ln 2
 HALF_PI = 1.5707963267948966      # double nearest pi/2
@@ -225,6 +226,7 @@ class Recipe:
     mask_kind: str        # "none", "causal", "window", "streaming"
     window: int = 0
     keep: int = 0         # streaming mask: initial tokens every later query sees
+    n_sel: int = 0        # > 0: decode over a selected key list of this length per (n, KV head)
     sink: str = "none"    # "none", "fixed", "normal"
     sink_values: tuple = ()
     bias: str = "none"    # "none" or "random10"
@@ -338,6 +340,24 @@ def bias_matrix(r: Recipe):
     return b.astype(np.float32)
 
 
+def key_index_set(r: Recipe) -> np.ndarray | None:
+    """(N, H, n_sel) int32 key lists, or None.  For each (n, KV head) one uniform
+    draw per cached key; the n_sel keys with the largest draws, in decreasing
+    draw order.  That is a uniformly random n_sel-subset in random order, the
+    shape of a top-k selection's output (positions scattered over the cache,
+    not sorted).  n_sel > S repeats the list cyclically."""
+    if r.n_sel <= 0:
+        return None
+    key = stream_key(r.seed, STREAM_KEY_INDEX)
+    out = np.empty((r.N, r.H, r.n_sel), dtype=np.int32)
+    for n in range(r.N):
+        for h in range(r.H):
+            u = uniform_f64(key, (n * r.H + h) * r.S, r.S)
+            order = np.argsort(-u, kind="stable")
+            out[n, h] = np.resize(order, r.n_sel)
+    return out
+
+
 def generate(r: Recipe) -> dict:
     """Whole workload on the host (numpy).  bf16 tensors are uint16 bit arrays."""
     out = {}
@@ -350,6 +370,7 @@ def generate(r: Recipe) -> dict:
         out[t] = arr
     out["sink"] = sink_logits(r)
     out["bias"] = bias_matrix(r)
+    out["key_idx"] = key_index_set(r)
     return out
 
 

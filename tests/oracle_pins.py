@@ -375,10 +375,71 @@ def check_streaming_mask(seed=14):
             assert np.allclose(full, comp, atol=1e-13) and np.allclose(lf, lc, atol=1e-13), (mode, W, keep)
 
 
+def check_index_set(seed=15):
+    """Exact attention over a key list: the full list in order is the dense
+    forward; a subset equals the dense forward with -inf added off the subset;
+    list order does not matter; a key listed twice equals the dense forward with
+    ln 2 added to its logit; entries outside [0, S) select nothing; one selected
+    key gives its value row and its own logit as lse (closed form)."""
+    rng = np.random.default_rng(seed)
+    N, H, Hq, L, S, E, Ev = 2, 2, 4, 3, 40, 5, 4
+    q, k, v = _rand(rng, N, Hq, L, E), _rand(rng, N, H, S, E), _rand(rng, N, H, S, Ev)
+    sink = rng.standard_normal(Hq)
+    bias = np.where(rng.random((L, S)) < 0.1, -np.inf, 0.0)
+    scale = 0.45
+    for mk, W in (("none", 0), ("causal", 0), ("window", 9)):
+        full = np.broadcast_to(np.arange(S), (N, H, S))
+        a = orc.attention_over_index_set(q, k, v, full, scale=scale, sink=sink, mask_kind=mk, window=W, bias=bias)
+        b = orc.attention_forward(q, k, v, scale=scale, sink=sink, mask_kind=mk, window=W, bias=bias)
+        assert np.allclose(a[0], b[0], atol=1e-13) and np.allclose(a[1], b[1], atol=1e-13), mk
+        # subsets with the last cached keys included (visible to every row under the masks)
+        idx = np.stack([np.stack([rng.permutation(S - 1)[:11] for _ in range(H)]) for _ in range(N)])
+        idx[..., 0] = S - 1  # distinct from the rest, which come from 0..S-2
+        dup = idx.copy()
+        dup[..., 1] = dup[..., 0]  # key S-1 listed twice
+        for lst, extra in ((idx, 0.0), (dup, math.log(2.0))):
+            got_o, got_l = orc.attention_over_index_set(q, k, v, lst, scale=scale, sink=sink, mask_kind=mk,
+                                                        window=W, bias=bias)
+            for n in range(N):
+                for hq in range(Hq):
+                    kvh = hq // (Hq // H)
+                    add = np.full(S, -np.inf)
+                    add[np.unique(lst[n, kvh])] = 0.0
+                    add[S - 1] += extra
+                    brow = bias + add[None, :]
+                    ref_o, ref_l = orc.attend_rows(q[n, hq], np.arange(L), k[n, kvh], v[n, kvh], L, scale=scale,
+                                                   sink=float(sink[hq]), mask_kind=mk, window=W, bias_rows=brow)
+                    assert np.allclose(got_o[n, hq], ref_o, atol=1e-13), (mk, n, hq, extra)
+                    assert np.allclose(got_l[n, hq], ref_l, atol=1e-13), (mk, n, hq, extra)
+        perm = idx[..., rng.permutation(idx.shape[-1])]
+        p_o, p_l = orc.attention_over_index_set(q, k, v, perm, scale=scale, sink=sink, mask_kind=mk, window=W)
+        i_o, i_l = orc.attention_over_index_set(q, k, v, idx, scale=scale, sink=sink, mask_kind=mk, window=W)
+        assert np.allclose(p_o, i_o, atol=1e-13) and np.allclose(p_l, i_l, atol=1e-13)
+    # entries outside [0, S) select nothing
+    pad = np.concatenate([np.full((N, H, 3), -1), idx, np.full((N, H, 2), S), np.full((N, H, 1), S + 7)], axis=-1)
+    a = orc.attention_over_index_set(q, k, v, pad, scale=scale, sink=sink)
+    b = orc.attention_over_index_set(q, k, v, idx, scale=scale, sink=sink)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    none = np.full((N, H, 4), -3)
+    o0, l0 = orc.attention_over_index_set(q, k, v, none, scale=scale)
+    assert np.all(o0 == 0.0) and np.all(l0 == -np.inf)
+    o1, l1 = orc.attention_over_index_set(q, k, v, none, scale=scale, sink=sink)
+    assert np.all(o1 == 0.0) and np.allclose(l1, np.broadcast_to(sink[None, :, None], l1.shape))
+    # one selected key: out = its value row, lse = its logit (closed form, no softmax code involved)
+    one = np.full((N, H, 1), 17)
+    o, l = orc.attention_over_index_set(q, k, v, one, scale=scale)
+    for n in range(N):
+        for hq in range(Hq):
+            kvh = hq // (Hq // H)
+            assert np.allclose(o[n, hq], np.broadcast_to(v[n, kvh, 17], (L, Ev)), atol=1e-15)
+            z = scale * sum(q[n, hq, :, e] * k[n, kvh, 17, e] for e in range(E))
+            assert np.allclose(l[n, hq], z, atol=1e-13)
+
+
 ALL_CHECKS = [
     check_dot_matches_sdpa, check_brute_force, check_rbf_expansion, check_rbf_limits,
     check_dot_limits, check_uniform_entropy_golden, check_sink_limit, check_sink_mass,
     check_zero_sink_equivalence, check_convexity, check_causal_alignment_golden,
     check_fully_masked_rows, check_window_semantics, check_permutation_equivariance,
-    check_gqa_repeat, check_streaming_mask,
+    check_gqa_repeat, check_streaming_mask, check_index_set,
 ]

@@ -64,7 +64,31 @@ def _lse_without_sink(z, vis, sink):
     return alpha, ps, lse0 if sink is not None else lse
 
 
+_real_select = orc.select_keys
+_real_visible_at = orc.visible_at
+
+
+def _select_unique(sel, S):
+    return np.unique(_real_select(sel, S))  # drops repeated listings
+
+
+def _select_clipped(sel, S):
+    return np.clip(np.asarray(sel, dtype=np.int64), 0, S - 1)  # clips padding instead of dropping it
+
+
+def _visible_at_list_position(rows, positions, S, L, mask_kind, window=0):
+    return _real_visible(rows, S, L, mask_kind, window)[:, np.arange(len(positions))]
+
+
+def _select_ignored(sel, S):
+    return np.arange(S)  # attends over the whole cache
+
+
 MUTATIONS = [
+    ("select_keys", _select_unique, pins.check_index_set),
+    ("select_keys", _select_clipped, pins.check_index_set),
+    ("select_keys", _select_ignored, pins.check_index_set),
+    ("visible_at", _visible_at_list_position, pins.check_index_set),
     ("logits", _rbf_direct_frame, pins.check_zero_sink_equivalence),
     ("logits", _rbf_direct_frame, pins.check_rbf_expansion),
     ("logits", _rbf_sign_flip, pins.check_rbf_limits),

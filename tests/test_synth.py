@@ -107,3 +107,23 @@ def test_recipe_table():
     assert len(names) == 6
     for r in sw.RECIPES.values():
         assert r.Hq % r.H == 0 and r.E in (64, 128) and r.Ev in (64, 128)
+
+
+def test_key_index_set_is_a_random_subset():
+    """Each (n, KV head) list holds n_sel distinct positions in [0, S), not sorted,
+    differs across heads, and repeats cyclically when n_sel > S."""
+    import dataclasses
+    base = sw.RECIPES["tiny_rbf_sink_causal_f32"]
+    r = dataclasses.replace(base, N=2, H=3, Hq=3, S=500, n_sel=37)
+    a, b = sw.key_index_set(r), sw.key_index_set(r)
+    assert a.shape == (2, 3, 37) and a.dtype == np.int32 and np.array_equal(a, b)
+    for n in range(2):
+        for h in range(3):
+            lst = a[n, h]
+            assert len(set(lst.tolist())) == 37 and lst.min() >= 0 and lst.max() < 500
+            assert not np.all(np.diff(lst) > 0)
+    assert not np.array_equal(a[0, 0], a[0, 1])
+    big = sw.key_index_set(dataclasses.replace(r, S=10, n_sel=25))
+    assert np.array_equal(big[0, 0, :10], big[0, 0, 10:20])
+    assert sorted(big[0, 0, :10].tolist()) == list(range(10))
+    assert sw.key_index_set(base) is None

@@ -48,6 +48,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_fwd.restype = ci
     lib.attn_fwd_streaming.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp, ci, vp]
     lib.attn_fwd_streaming.restype = ci
+    lib.attn_decode_indexed.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, ci, cf, vp, ci, ci, vp,
+                                        vp]
+    lib.attn_decode_indexed.restype = ci
     lib.attn_status_string.argtypes = [ci]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_release_workspace.argtypes = []
@@ -152,6 +155,61 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float,
             st = lib.attn_fwd_streaming(*common, int(window), int(keep_first), *tail)
         else:
             st = lib.attn_fwd(*common, MASKS[mask_kind], int(window), *tail)
+    _check(st)
+    return out, lse
+
+
+def attn_decode_indexed_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, idx_ptr, n_sel, N, Hq, H, L, S, E, Ev, scale,
+                            sink_ptr, mask_kind, window, bias_ptr, stream_ptr) -> int:
+    """The index-set decode entry point with integer pointers; returns the status code."""
+    lib = load_library()
+    c = lambda p: None if p is None else ctypes.c_void_p(int(p))  # noqa: E731
+    return lib.attn_decode_indexed(c(q_ptr), c(k_ptr), c(v_ptr), c(out_ptr), c(lse_ptr), c(idx_ptr), int(n_sel),
+                                   int(N), int(Hq), int(H), int(L), int(S), int(E), int(Ev), float(scale),
+                                   c(sink_ptr), int(mask_kind), int(window), c(bias_ptr), c(stream_ptr))
+
+
+def attn_decode_indexed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, key_idx: torch.Tensor, *, scale: float,
+                        sink: torch.Tensor | None = None, mask_kind: str = "none", window: int = 0,
+                        bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                        lse: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None):
+    """Exact decode attention over listed keys.  Returns (out, lse).
+
+    q (N, Hq, L, E), k (N, H, S, E), v (N, H, S, Ev): contiguous bfloat16 CUDA
+    tensors with (Hq/H)*L <= 16.  key_idx (N, H, n_sel) int32 CUDA tensor of key
+    positions; entries outside [0, S) select nothing.  sink, bias, mask_kind
+    ("none", "causal", "window") and window as in attn_fwd.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v), ("key_idx", key_idx)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4 or key_idx.dim() != 3:
+        raise ValueError("q, k, v must be 4-D and key_idx 3-D")
+    if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must be bfloat16")
+    if key_idx.dtype != torch.int32:
+        raise ValueError("key_idx must be int32")
+    N, Hq, L, E = q.shape
+    _, H, S, _ = k.shape
+    Ev = v.shape[3]
+    if tuple(key_idx.shape[:2]) != (N, H):
+        raise ValueError("key_idx must be (N, H, n_sel)")
+    if sink is not None and (sink.dtype != torch.float32 or sink.numel() != Hq or not sink.is_cuda
+                             or not sink.is_contiguous()):
+        raise ValueError("sink must be a contiguous CUDA float32 tensor of Hq values")
+    if bias is not None and (bias.dtype != torch.float32 or tuple(bias.shape) != (L, S) or not bias.is_cuda
+                             or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous CUDA float32 (L, S) tensor")
+    if out is None:
+        out = torch.empty((N, Hq, L, Ev), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((N, Hq, L), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = load_library().attn_decode_indexed(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(key_idx), key_idx.shape[2], N, Hq, H, L, S, E, Ev,
+            float(scale), _ptr(sink), MASKS[mask_kind], int(window), _ptr(bias), ctypes.c_void_p(stream.cuda_stream))
     _check(st)
     return out, lse
 

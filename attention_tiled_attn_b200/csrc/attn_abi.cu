@@ -100,11 +100,9 @@ int ensure_workspace(int dev, size_t bytes, cudaStream_t stream, void** out) {
 
 }  // namespace
 
-// Shared by the public entry points once they have checked their mask arguments:
-// validates the rest and dispatches (fp32 kernel, split-key decode, tcgen05 prefill).
-int forward(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L, int S,
-            int E, int Ev, float scale, int mode, const float* sink_logits, int mask_kind, int window, int keep,
-            const float* bias, int dtype, void* stream_ptr) {
+// Checks shared by every entry point (after each has checked its mask arguments).
+int validate(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L, int S,
+             int E, int Ev, float scale, int mode, const float* sink_logits, const float* bias, int dtype) {
   if (!q || !k || !v || !out) return ATTN_ERR_NULL_POINTER;
   if (N < 1 || Hq < 1 || H < 1 || L < 1 || S < 1) return ATTN_ERR_BAD_SHAPE;
   if (Hq % H != 0) return ATTN_ERR_GQA;
@@ -124,11 +122,12 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
   if (bias && !aligned(bias, 16)) return ATTN_ERR_ALIGNMENT;
   if (lse && !aligned(lse, 4)) return ATTN_ERR_ALIGNMENT;
   if (sink_logits && !aligned(sink_logits, 4)) return ATTN_ERR_ALIGNMENT;
+  return ATTN_OK;
+}
 
-  int dev = 0, sms = 0, major = 0;
-  if (device_info(&dev, &sms, &major) != ATTN_OK) return ATTN_ERR_CUDA;
-  if (major != 10) return ATTN_ERR_DEVICE;
-
+AttnArgs make_args(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L,
+                   int S, int E, int Ev, float scale, int mode, const float* sink_logits, int mask_kind, int window,
+                   int keep, const float* bias) {
   AttnArgs a{};
   a.q = q;
   a.k = k;
@@ -149,6 +148,21 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
   a.window = window;
   a.keep = keep;
   a.bias = bias;
+  return a;
+}
+
+// Shared by the public entry points once they have checked their mask arguments:
+// validates the rest and dispatches (fp32 kernel, split-key decode, tcgen05 prefill).
+int forward(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L, int S,
+            int E, int Ev, float scale, int mode, const float* sink_logits, int mask_kind, int window, int keep,
+            const float* bias, int dtype, void* stream_ptr) {
+  const int st = validate(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, bias, dtype);
+  if (st != ATTN_OK) return st;
+  int dev = 0, sms = 0, major = 0;
+  if (device_info(&dev, &sms, &major) != ATTN_OK) return ATTN_ERR_CUDA;
+  if (major != 10) return ATTN_ERR_DEVICE;
+  const AttnArgs a =
+      make_args(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, mask_kind, window, keep, bias);
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
 
   if (dtype == ATTN_FP32) return launch_fp32(a, stream);
@@ -182,6 +196,31 @@ int attn_fwd_streaming(const void* q, const void* k, const void* v, void* out, f
   if (keep_first < 0) return ATTN_ERR_KEEP;
   return attn::forward(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, attn::MASK_STREAM,
                        window, keep_first, bias, dtype, stream_ptr);
+}
+
+int attn_decode_indexed(const void* q, const void* k, const void* v, void* out, float* lse, const int* key_idx,
+                        int n_sel, int N, int Hq, int H, int L, int S, int E, int Ev, float scale,
+                        const float* sink_logits, int mask_kind, int window, const float* bias, void* stream_ptr) {
+  using namespace attn;
+  if (!key_idx) return ATTN_ERR_NULL_POINTER;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_SLIDING_WINDOW) return ATTN_ERR_MASK;
+  if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window < 1) return ATTN_ERR_WINDOW;
+  int st = validate(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, ATTN_DOT, sink_logits, bias, ATTN_BF16);
+  if (st != ATTN_OK) return st;
+  if (n_sel < 1 || static_cast<long long>(N) * H * n_sel > (1LL << 40)) return ATTN_ERR_BAD_SHAPE;
+  if (!aligned(key_idx, 4)) return ATTN_ERR_ALIGNMENT;
+  if ((Hq / H) * L > 16) return ATTN_ERR_NOT_DECODE;
+  int dev = 0, sms = 0, major = 0;
+  if (device_info(&dev, &sms, &major) != ATTN_OK) return ATTN_ERR_CUDA;
+  if (major != 10) return ATTN_ERR_DEVICE;
+  const AttnArgs a =
+      make_args(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, ATTN_DOT, sink_logits, mask_kind, window, 0, bias);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  void* ws = nullptr;
+  const size_t need = decode_gather_workspace_bytes(a, n_sel, sms);
+  st = ensure_workspace(dev, need, stream, &ws);
+  if (st != ATTN_OK) return st;
+  return launch_decode_gather_bf16(a, key_idx, n_sel, ws, need, sms, stream);
 }
 
 const char* attn_status_string(int status) {

@@ -21,6 +21,16 @@
 //
 // Masks follow the bottom-right alignment of page "SDPA란 무엇인가" §4
 // (trap 3): query i of L sits at key position i + S - L.
+//
+// GATHER variant: exact attention over a listed key subset (page "기술 요약:
+// SOCKET - 희소 어텐션을 위한 SOft Collision Kernel EsTimator", 방법론, step 4:
+// top-k keys are selected, then exact attention runs on them).  A unit's chunks
+// are 64 consecutive list entries; the producer warp gathers the listed K and
+// V rows with 16-byte cp.async copies (two whole 256-byte rows per warp
+// instruction at E = 128, four warps) into the same swizzled stage layout, and stores the
+// chunk's key positions in shared memory for the consumers' masks.  The list
+// entries are loaded two chunks ahead.  (One bulk copy per row through the TMA
+// engine measured half the throughput: at 256 bytes its per-copy cost dominates.)
 
 #include <cstdint>
 #include <cuda.h>
@@ -37,6 +47,9 @@ namespace {
 constexpr int DC = 64;             // keys per chunk
 constexpr int DWARPS = 4;          // consumer warps (16 keys each)
 constexpr int DTHREADS = (DWARPS + 1) * 32;
+// GATHER: producer warps, each issuing every GWARPS-th copy instruction of a chunk.  One warp
+// keeps too few copies in flight for random rows; 4 measured best (5 and 6 were slower).
+constexpr int GWARPS = 4;
 constexpr float D_RESCALE_THRESHOLD = 8.0f;
 
 struct DecodeParams {  // 128 bytes: kept at that size, the kernels' code generation depends on it
@@ -60,16 +73,27 @@ struct DecodeParams {  // 128 bytes: kept at that size, the kernels' code genera
 };
 static_assert(sizeof(DecodeParams) == 128, "DecodeParams layout");
 
-template <int E, int EV>
+// GATHER only: the key lists and the K/V base pointers (a separate kernel argument,
+// so the other variants' parameter block stays as it is)
+struct GatherArgs {
+  const int* idx;            // [N*H][n_sel] key positions
+  const __nv_bfloat16* k;    // [N*H][S][E]
+  const __nv_bfloat16* v;    // [N*H][S][Ev]
+  int n_sel;
+};
+
+template <int E, int EV, bool GATHER = false>
 struct DCfg {
+  static constexpr int K_BYTES = DC * E * 2;  // V part of a stage starts here
   static constexpr int STAGE_BYTES = DC * (E + EV) * 2;
-  static constexpr int NSTAGE = (E + EV >= 256) ? 5 : 8;
+  static constexpr int NSTAGE = (E + EV >= 256) ? 5 : (GATHER ? 7 : 8);
   static constexpr int OFF_STAGES = 0;
   static constexpr int OFF_MERGE = NSTAGE * STAGE_BYTES;              // [DWARPS][16][EV] f32
   static constexpr int OFF_ML = OFF_MERGE + DWARPS * 16 * EV * 4;     // [DWARPS][16][2] f32
   static constexpr int OFF_BAR = OFF_ML + DWARPS * 16 * 2 * 4;
   static constexpr int OFF_MISC = OFF_BAR + 2 * NSTAGE * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int OFF_KEYS = OFF_MISC + 16;                      // [NSTAGE][DC] int (GATHER)
+  static constexpr int SMEM_BYTES = OFF_KEYS + (GATHER ? NSTAGE * DC * 4 : 0) + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -101,6 +125,18 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// 16-byte global -> shared copy through L2 only
+// 16-byte global -> shared copy through L2 only
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// arrive on an mbarrier once this thread's earlier cp.async copies have landed;
+// the arrival counts toward the barrier's expected count
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(DWARPS * 32) : "memory"); }
 
 // byte offset of (row, 16-byte chunk c) inside a swizzled chunk buffer of 64-row, 128-byte boxes
@@ -108,11 +144,11 @@ __device__ __forceinline__ uint32_t sw_off(int row, int c16) {
   return (c16 >> 3) * (DC * 128) + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
 }
 
-template <int E, int EV, bool STREAM>
-__global__ void __launch_bounds__(DTHREADS, 1)
+template <int E, int EV, bool STREAM, bool GATHER>
+__global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
     decode_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                          const DecodeParams p) {
-  using C = DCfg<E, EV>;
+                          const DecodeParams p, const GatherArgs ga) {
+  using C = DCfg<E, EV, GATHER>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t sb = (raw_addr + 1023u) & ~1023u;
@@ -129,7 +165,8 @@ __global__ void __launch_bounds__(DTHREADS, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int s = 0; s < C::NSTAGE; ++s) {
-      mbar_init(full_bar(s), 1);
+      // GATHER: each producer lane arrives twice, once when its copies land and once for its key positions
+      mbar_init(full_bar(s), GATHER ? 64 * GWARPS : 1);
       mbar_init(empty_bar(s), DWARPS);
     }
     fence_barrier_init();
@@ -137,6 +174,70 @@ __global__ void __launch_bounds__(DTHREADS, 1)
   __syncthreads();
   if (c_end <= c_begin) return;
 
+  if (GATHER && warp >= DWARPS) {
+    const int pw = warp - DWARPS;  // this warp issues copy instructions pw, pw + GWARPS, ...
+    // ---------------- gathering producer (whole warp) ----------------
+    int* keys_s = reinterpret_cast<int*>(sp + C::OFF_KEYS);
+    // the list entries of chunk c: lane l holds entries l and l + 32 (-1 past the list's end);
+    // they are loaded two chunks ahead so their latency overlaps earlier chunks' copies
+    auto load_list = [&](long long c, int& a, int& b) {
+      const long long u = c / p.nc;
+      const int local = static_cast<int>(c % p.nc);
+      const int* lst = ga.idx + static_cast<size_t>(u) * ga.n_sel + static_cast<size_t>(local) * DC;
+      const int n_here = min(DC, ga.n_sel - local * DC);
+      a = lane < n_here ? __ldg(lst + lane) : -1;
+      b = lane + 32 < n_here ? __ldg(lst + lane + 32) : -1;
+    };
+    constexpr int PK = E / 8, RK = 32 / PK;  // 16-byte pieces per K row, K rows per warp instruction
+    constexpr int PV = EV / 8, RV = 32 / PV;
+    int na0 = -1, na1 = -1, nb0 = -1, nb1 = -1;  // chunks c + 1 and c + 2
+    if (c_begin < c_end) load_list(c_begin, na0, na1);
+    if (c_begin + 1 < c_end) load_list(c_begin + 1, nb0, nb1);
+    for (long long c = c_begin; c < c_end; ++c) {
+      const int idx = static_cast<int>(c - c_begin);
+      const int s = idx % C::NSTAGE;
+      const uint32_t ph = (idx / C::NSTAGE) & 1;
+      int j0 = na0, j1 = na1;
+      na0 = nb0;
+      na1 = nb1;
+      if (c + 2 < c_end) load_list(c + 2, nb0, nb1);
+      const bool w_ok = mbar_wait(empty_bar(s), ph ^ 1);
+      if (!__all_sync(0xffffffffu, w_ok) || *abort_flag) {
+        if (lane == 0) *abort_flag = 1;
+        break;
+      }
+      const long long u = c / p.nc;
+      j0 = (j0 >= 0 && j0 < p.S) ? j0 : -1;  // entries outside [0, S) select nothing
+      j1 = (j1 >= 0 && j1 < p.S) ? j1 : -1;
+      if (pw == 0) {
+        keys_s[s * DC + lane] = j0;
+        keys_s[s * DC + 32 + lane] = j1;
+      }
+      const __nv_bfloat16* kb = ga.k + static_cast<size_t>(u) * p.S * E;
+      const __nv_bfloat16* vb = ga.v + static_cast<size_t>(u) * p.S * EV;
+      const uint32_t kdst = sb + C::OFF_STAGES + s * C::STAGE_BYTES;
+      const uint32_t vdst = kdst + C::K_BYTES;
+      // rows without a key (padding) copy row 0 of the unit; the consumers mask them
+#pragma unroll 4
+      for (int m = pw; m < DC / RK; m += GWARPS) {
+        const int r = m * RK + lane / PK;  // rows of one instruction are all below 32 or all above
+        const int jr = __shfl_sync(0xffffffffu, m * RK < 32 ? j0 : j1, r & 31);
+        const int col = lane % PK;
+        cp_async16(kdst + sw_off(r, col), kb + static_cast<size_t>(jr < 0 ? 0 : jr) * E + col * 8);
+      }
+#pragma unroll 4
+      for (int m = pw; m < DC / RV; m += GWARPS) {
+        const int r = m * RV + lane / PV;
+        const int jr = __shfl_sync(0xffffffffu, m * RV < 32 ? j0 : j1, r & 31);
+        const int col = lane % PV;
+        cp_async16(vdst + sw_off(r, col), vb + static_cast<size_t>(jr < 0 ? 0 : jr) * EV + col * 8);
+      }
+      cp_async_mbar_arrive(full_bar(s));
+      mbar_arrive(full_bar(s));  // releases this lane's key positions
+    }
+    cp_async_wait_all();  // no copy may still be in flight at exit
+    return;
+  }
   if (warp == DWARPS) {
     // ---------------- producer ----------------
     if (lane == 0) {
@@ -283,9 +384,10 @@ __global__ void __launch_bounds__(DTHREADS, 1)
       break;
     }
     const uint32_t kbuf = sb + C::OFF_STAGES + s * C::STAGE_BYTES;
-    const uint32_t vbuf = kbuf + E * DC * 2;
+    const uint32_t vbuf = kbuf + C::K_BYTES;
     const int j0 = warp * 16;  // this warp's keys within the chunk
-    const int key0 = chunk_key0<STREAM>(p, static_cast<int>(c % p.nc)) + j0;
+    const int key0 = GATHER ? 0 : chunk_key0<STREAM>(p, static_cast<int>(c % p.nc)) + j0;
+    const int* keys_c = reinterpret_cast<const int*>(sp + C::OFF_KEYS) + s * DC + j0;  // GATHER
 
     // S = Q K^T for 16 keys (two n-tiles of 8)
     float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -301,7 +403,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
       }
     }
     // logits in base 2, masks and bias
-    const bool need_mask = p.mask_kind != MASK_NONE || p.bias != nullptr || key0 + 16 > p.S;
+    const bool need_mask = GATHER || p.mask_kind != MASK_NONE || p.bias != nullptr || key0 + 16 > p.S;
 #pragma unroll
     for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -309,13 +411,15 @@ __global__ void __launch_bounds__(DTHREADS, 1)
         const int h = e >> 1;
         float zz = sc[t][e] * p.c_dot;
         if (need_mask) {
-          const int key = key0 + t * 8 + cq + (e & 1);
-          if constexpr (STREAM) {
+          const int key = GATHER ? keys_c[t * 8 + cq + (e & 1)] : key0 + t * 8 + cq + (e & 1);
+          if constexpr (GATHER) {
+            if (key < 0 || key < lo_r[h] || key >= hi_r[h]) zz = -INFINITY;  // -1: no key listed here
+          } else if constexpr (STREAM) {
             if (key >= hi_r[h] || (key < lo_r[h] && key >= p.keep)) zz = -INFINITY;
           } else {
             if (key < lo_r[h] || key >= hi_r[h]) zz = -INFINITY;
           }
-          if (p.bias != nullptr && live_r[h] && key < p.S)
+          if (p.bias != nullptr && live_r[h] && key >= 0 && key < p.S)
             zz = fmaf(p.bias[static_cast<size_t>((rA + 8 * h) % p.L) * p.S + key], LOG2E, zz);
         }
         sc[t][e] = zz;
@@ -418,6 +522,22 @@ struct DecodePlan {
   long long T;
 };
 
+// the even split of T chunks over a persistent grid, shared by both plans
+void split(DecodePlan& d, const AttnArgs& a, int num_sms) {
+  d.T = static_cast<long long>(a.N) * a.H * d.nc;
+  d.G = static_cast<int>(d.T < num_sms ? d.T : num_sms);
+  const long long per = (d.T + d.G - 1) / d.G;
+  d.max_segs = static_cast<int>((per + d.nc - 1) / d.nc + 1);
+}
+
+// GATHER: a unit's chunks are 64 consecutive entries of its key list
+DecodePlan plan_gather(const AttnArgs& a, int n_sel, int num_sms) {
+  DecodePlan d{};
+  d.nc = (n_sel + DC - 1) / DC;
+  split(d, a, num_sms);
+  return d;
+}
+
 DecodePlan plan(const AttnArgs& a, int num_sms) {
   DecodePlan d{};
   const int off = a.S - a.L;
@@ -440,23 +560,23 @@ DecodePlan plan(const AttnArgs& a, int num_sms) {
     }
   }
   d.nc = d.nc_head + (kb_hi - d.kb_win);
-  d.T = static_cast<long long>(a.N) * a.H * d.nc;
-  d.G = static_cast<int>(d.T < num_sms ? d.T : num_sms);
-  const long long per = (d.T + d.G - 1) / d.G;
-  d.max_segs = static_cast<int>((per + d.nc - 1) / d.nc + 1);
+  split(d, a, num_sms);
   return d;
 }
 
-template <int E, int EV, bool STREAM>
-int launch_decode_impl(const AttnArgs& a, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream) {
-  using C = DCfg<E, EV>;
-  const DecodePlan d = plan(a, num_sms);
+template <int E, int EV, bool STREAM, bool GATHER>
+int launch_decode_impl(const AttnArgs& a, const GatherArgs& ga, void* ws, size_t ws_bytes, int num_sms,
+                       cudaStream_t stream) {
+  using C = DCfg<E, EV, GATHER>;
+  const DecodePlan d = GATHER ? plan_gather(a, ga.n_sel, num_sms) : plan(a, num_sms);
   const size_t slots = static_cast<size_t>(d.G) * d.max_segs;
   const size_t need = slots * 16 * (EV + 2) * sizeof(float);
   if (ws_bytes < need) return -12;
-  CUtensorMap tk, tv;
-  if (!make_map_rows(&tk, a.k, E, a.S, static_cast<long long>(a.N) * a.H, DC)) return -13;
-  if (!make_map_rows(&tv, a.v, EV, a.S, static_cast<long long>(a.N) * a.H, DC)) return -13;
+  CUtensorMap tk{}, tv{};  // GATHER reads K and V through plain pointers; its maps stay unused
+  if (!GATHER) {
+    if (!make_map_rows(&tk, a.k, E, a.S, static_cast<long long>(a.N) * a.H, DC)) return -13;
+    if (!make_map_rows(&tv, a.v, EV, a.S, static_cast<long long>(a.N) * a.H, DC)) return -13;
+  }
   DecodeParams p{};
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.out = static_cast<__nv_bfloat16*>(a.out);
@@ -483,10 +603,10 @@ int launch_decode_impl(const AttnArgs& a, void* ws, size_t ws_bytes, int num_sms
   p.G = d.G;
   p.max_segs = d.max_segs;
   p.c_dot = a.scale * LOG2E;
-  auto kern = decode_partial_kernel<E, EV, STREAM>;
+  auto kern = decode_partial_kernel<E, EV, STREAM, GATHER>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return -13;
-  kern<<<d.G, DTHREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+  kern<<<d.G, GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, C::SMEM_BYTES, stream>>>(tk, tv, p, ga);
   if (cudaGetLastError() != cudaSuccess) return -13;
   decode_combine_kernel<EV><<<a.N * a.H, 128, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? 0 : -13;
@@ -503,13 +623,37 @@ size_t decode_workspace_bytes(const AttnArgs& a, int num_sms) {
   return static_cast<size_t>(d.G) * d.max_segs * 16 * (a.Ev + 2) * sizeof(float);
 }
 
+size_t decode_gather_workspace_bytes(const AttnArgs& a, int n_sel, int num_sms) {
+  const DecodePlan d = plan_gather(a, n_sel, num_sms);
+  return static_cast<size_t>(d.G) * d.max_segs * 16 * (a.Ev + 2) * sizeof(float);
+}
+
+int launch_decode_gather_bf16(const AttnArgs& a, const int* key_idx, int n_sel, void* ws, size_t ws_bytes,
+                              int num_sms, cudaStream_t stream) {
+  GatherArgs ga{};
+  ga.idx = key_idx;
+  ga.k = static_cast<const __nv_bfloat16*>(a.k);
+  ga.v = static_cast<const __nv_bfloat16*>(a.v);
+  ga.n_sel = n_sel;
+#define ATTN_GATHER_CASE(e, ev) \
+  if (a.E == e && a.Ev == ev) return launch_decode_impl<e, ev, false, true>(a, ga, ws, ws_bytes, num_sms, stream);
+  ATTN_GATHER_CASE(128, 128)
+  ATTN_GATHER_CASE(64, 64)
+  ATTN_GATHER_CASE(64, 128)
+  ATTN_GATHER_CASE(128, 64)
+#undef ATTN_GATHER_CASE
+  return -4;
+}
+
 int launch_decode_bf16(const AttnArgs& a, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream) {
   // kept initial keys need the streaming mask test even where the plan makes no
   // head/window split (kept keys and window overlap: nc_head is then 0)
   const bool st = a.mask_kind == MASK_STREAM && a.keep > 0;
-#define ATTN_DECODE_CASE(e, ev)                                                       \
-  if (a.E == e && a.Ev == ev) return st ? launch_decode_impl<e, ev, true>(a, ws, ws_bytes, num_sms, stream) \
-                                        : launch_decode_impl<e, ev, false>(a, ws, ws_bytes, num_sms, stream);
+  const GatherArgs none{};
+#define ATTN_DECODE_CASE(e, ev)                                                                          \
+  if (a.E == e && a.Ev == ev)                                                                            \
+    return st ? launch_decode_impl<e, ev, true, false>(a, none, ws, ws_bytes, num_sms, stream)           \
+              : launch_decode_impl<e, ev, false, false>(a, none, ws, ws_bytes, num_sms, stream);
   ATTN_DECODE_CASE(128, 128)
   ATTN_DECODE_CASE(64, 64)
   ATTN_DECODE_CASE(64, 128)

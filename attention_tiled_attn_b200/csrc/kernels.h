@@ -37,6 +37,11 @@ int launch_fp32(const AttnArgs& a, cudaStream_t stream);
 // Decode (bf16, (Hq/H) * L <= 16): key-split partial kernel + combine kernel.
 bool decode_eligible(const AttnArgs& a);
 size_t decode_workspace_bytes(const AttnArgs& a, int num_sms);
+// Decode over listed keys: key_idx [N*H][n_sel] device array of key positions
+// (entries outside [0, S) select nothing); same workspace scheme.
+size_t decode_gather_workspace_bytes(const AttnArgs& a, int n_sel, int num_sms);
+int launch_decode_gather_bf16(const AttnArgs& a, const int* key_idx, int n_sel, void* workspace,
+                              size_t workspace_bytes, int num_sms, cudaStream_t stream);
 int launch_decode_bf16(const AttnArgs& a, void* workspace, size_t workspace_bytes, int num_sms,
                        cudaStream_t stream);
 

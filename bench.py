@@ -48,11 +48,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dominant kernel from one ncu capture of the same kernel build; the capture
 # command and counters are in profiles/.  Must be reset when the kernel changes.
 NCU_TRAFFIC_BYTES = {
-    "dot_causal_2k_bf16": 132_793_088 + 13_932_032,          # prefill_kernel<128,128,dot>
-    "sink_gqa_window_16k_bf16": 167_958_528 + 100_350_976,   # prefill_kernel<64,64,dot>
-    "rbf_registers_4k_bf16": 37_890_048 + 91_904,            # prefill_kernel<64,64,rbf>
-    # decode_partial_kernel<128,128>: batch-2 capture (1.0738e9 + 4.43e6 B) scaled by 16 to batch 32
-    "decode_sink_gqa_128k_bf16": 16 * (1_073_818_000 + 4_434_432),
+    "dot_causal_2k_bf16": 129_022_720 + 11_566_848,          # prefill_kernel<128,128,dot>
+    "sink_gqa_window_16k_bf16": 167_928_576 + 98_604_032,    # prefill_kernel<64,64,dot>
+    "rbf_registers_4k_bf16": 37_884_672 + 392_192,           # prefill_kernel<64,64,rbf>
+    # decode_partial_kernel<128,128>: batch-2 capture scaled by 16 to batch 32
+    "decode_sink_gqa_128k_bf16": 16 * (1_073_819_648 + 6_067_200),
+    # the same kernel's gather variant over 3971 listed keys (--select 3971), batch-2 capture scaled by 16
+    "decode_sink_gqa_128k_bf16:select3971": 16 * (32_867_072 + 5_376),
 }
 
 
@@ -99,6 +101,9 @@ def decode_keys(r: sw.Recipe) -> int:
 
 def work_units(r: sw.Recipe):
     """(amount, unit, roofline bound) of one step of workload r on one GPU."""
+    if r.n_sel > 0:
+        # listed-key decode: the gathered K and V rows plus the key lists themselves
+        return r.N * r.H * r.n_sel * ((r.E + r.Ev) * 2 + 4), "GB/s", "hbm"
     if is_decode(r):
         kv_bytes = r.N * r.H * decode_keys(r) * (r.E + r.Ev) * 2
         return kv_bytes, "GB/s", "hbm"
@@ -248,6 +253,11 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
     stream = torch.cuda.current_stream()
 
     def step():
+        if r.n_sel > 0:
+            attn.attn_decode_indexed(t["q"], t["k"], t["v"], t["key_idx"], scale=r.scale, sink=t["sink"],
+                                     mask_kind=r.mask_kind, window=r.window, bias=t["bias"], out=out, lse=lse,
+                                     stream=stream)
+            return
         attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=r.mode, sink=t["sink"], mask_kind=r.mask_kind,
                       window=r.window, keep_first=r.keep, bias=t["bias"], out=out, lse=lse, stream=stream)
 
@@ -274,7 +284,7 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
     else:
         peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         punit = "GB/s"
-    traffic = NCU_TRAFFIC_BYTES.get(name)
+    traffic = NCU_TRAFFIC_BYTES.get(name if r.n_sel == 0 else f"{name}:select{r.n_sel}")
     res = {
         "recipe": r, "amount": amount, "unit": unit, "secs_max": secs_max, "secs": secs,
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": punit,
@@ -296,8 +306,9 @@ def e2e_measure(res, steps, warmup):
     import attention_tiled_attn_b200 as attn
     r = res["recipe"]
     t = res["tensors"]
-    host = {k: t[k].cpu().pin_memory() for k in ("q", "k", "v")}
-    dev = {k: torch.empty_like(t[k]) for k in ("q", "k", "v")}
+    names = ("q", "k", "v", "key_idx") if r.n_sel > 0 else ("q", "k", "v")
+    host = {k: t[k].cpu().pin_memory() for k in names}
+    dev = {k: torch.empty_like(t[k]) for k in names}
     out_host = torch.empty(res["out"].shape, dtype=res["out"].dtype).pin_memory()
     lse_host = torch.empty(res["lse"].shape, dtype=torch.float32).pin_memory()
     stream = torch.cuda.current_stream()
@@ -305,11 +316,16 @@ def e2e_measure(res, steps, warmup):
     d2h = out_host.numel() * out_host.element_size() + lse_host.numel() * 4
 
     def step():
-        for k in ("q", "k", "v"):
+        for k in names:
             dev[k].copy_(host[k], non_blocking=True)
-        attn.attn_fwd(dev["q"], dev["k"], dev["v"], scale=r.scale, mode=r.mode, sink=t["sink"],
-                      mask_kind=r.mask_kind, window=r.window, keep_first=r.keep, bias=t["bias"], out=res["out"],
-                      lse=res["lse"], stream=stream)
+        if r.n_sel > 0:
+            attn.attn_decode_indexed(dev["q"], dev["k"], dev["v"], dev["key_idx"], scale=r.scale, sink=t["sink"],
+                                     mask_kind=r.mask_kind, window=r.window, bias=t["bias"], out=res["out"],
+                                     lse=res["lse"], stream=stream)
+        else:
+            attn.attn_fwd(dev["q"], dev["k"], dev["v"], scale=r.scale, mode=r.mode, sink=t["sink"],
+                          mask_kind=r.mask_kind, window=r.window, keep_first=r.keep, bias=t["bias"], out=res["out"],
+                          lse=res["lse"], stream=stream)
         out_host.copy_(res["out"], non_blocking=True)
         lse_host.copy_(res["lse"], non_blocking=True)
 
@@ -342,10 +358,12 @@ class OracleSample:
     """Runs the float64 oracle (as it stands) on row blocks of one (n, hq) head
     of workload r, and converts the time into the workload's unit."""
 
-    def __init__(self, r: sw.Recipe, n: int = 0, hq: int = 0):
+    def __init__(self, r: sw.Recipe, n: int = 0, hq: int = 0, key_idx=None):
         from oracle import attention as orc
         self.orc, self.r, self.hq = orc, r, hq
         kvh = hq // r.group
+        if r.n_sel > 0:  # the unit's key list (key_idx: the workload's lists, when already drawn)
+            self.key_list = (sw.key_index_set(r) if key_idx is None else key_idx)[n, kvh]
         self.q = sw.tensor_slice_f64(r, "q", n, hq)
         self.k = sw.tensor_slice_f64(r, "k", n, kvh)
         self.v = sw.tensor_slice_f64(r, "v", n, kvh)
@@ -357,10 +375,19 @@ class OracleSample:
 
     def rows_amount(self, rows):
         r = self.r
+        if r.n_sel > 0:
+            return work_units(r)[0] / (r.N * r.Hq) * rows.size / r.L
         return float(row_pairs(r, rows).sum()) * self.per_pair
 
     def run(self, rows):
         r = self.r
+        if r.n_sel > 0:
+            # the index-set oracle on this head's L rows (decode: L is small); rows counts the work done
+            self.orc.attention_over_index_set(
+                self.q[None, None], self.k[None, None], self.v[None, None], self.key_list[None, None],
+                scale=r.scale, sink=None if self.sink is None else np.array([self.sink]), mask_kind=r.mask_kind,
+                window=r.window, bias=self.bias)
+            return self.rows_amount(np.arange(r.L))
         for i0 in range(0, rows.size, 256):
             rr = rows[i0:i0 + 256]
             self.orc.attend_rows(self.q[rr], rr, self.k, self.v, r.L, scale=r.scale, mode=r.mode, sink=self.sink,
@@ -378,10 +405,11 @@ def cpu_baseline(r: sw.Recipe, budget_s: float = 12.0, wall_limit_s: float = 40.
     done, secs, blocks, heads = 0.0, 0.0, 0, 0
     unit = work_units(r)[1]
     t_start = time.perf_counter()
+    key_idx = sw.key_index_set(r)
     stop = False
     for n in range(r.N):
         for hq in range(r.Hq):
-            smp = OracleSample(r, n, hq)
+            smp = OracleSample(r, n, hq, key_idx)
             heads += 1
             for i1 in range(r.L, 0, -256):
                 rows = np.arange(max(0, i1 - 256), i1)
@@ -435,6 +463,8 @@ def ours(args):
             elif is_decode(r0):
                 runs.append((name + ":streaming_keep4_w4096",
                              dataclasses.replace(r0, mask_kind="streaming", window=4096, keep=4)))
+                # exact attention over a 33x-sparse key selection (S/33 keys per KV head, random positions)
+                runs.append((name + ":top_k_33x", dataclasses.replace(r0, n_sel=r0.S // 33)))
         for label, rr in runs:
             base = sw.RECIPES[rr.name]
             sw.RECIPES[rr.name] = rr
@@ -448,6 +478,7 @@ def ours(args):
                 "unit": res["unit"], "ms_per_step": round(res["secs_max"] / k * 1e3, 4),
                 "roofline_frac": res["roofline"]["frac"], "bound": res["roofline"]["bound"],
                 "mode": rr.mode, "sink": rr.sink != "none", "mask": rr.mask_kind,
+                **({"keys_listed_per_kv_head": rr.n_sel} if rr.n_sel > 0 else {}),
             }
             del res
             torch.cuda.empty_cache()
@@ -458,6 +489,9 @@ def ours(args):
                 if ctl in extra:
                     extra[label]["time_vs_" + ctl.split(":")[1]] = round(
                         extra[label]["ms_per_step"] / extra[ctl]["ms_per_step"], 4)
+            if label + ":top_k_33x" in extra:
+                extra[label + ":top_k_33x"]["time_vs_dense"] = round(
+                    extra[label + ":top_k_33x"]["ms_per_step"] / extra[label]["ms_per_step"], 4)
     if rank == 0:
         line = {
             "metric": METRIC,
@@ -472,7 +506,8 @@ def ours(args):
             "vs_baseline": None,
             "dtype": "bf16" if r.dtype == "bf16" else "f32",
             "data": "synthetic (seeded counter-based N(0,1) draws, see synth/workloads.py)",
-            "config": {"workload": r.name, "N": r.N, "Hq": r.Hq, "H": r.H, "L": r.L, "S": r.S, "E": r.E,
+            "config": {"workload": r.name, **({"keys_listed_per_kv_head": r.n_sel} if r.n_sel > 0 else {}),
+                       "N": r.N, "Hq": r.Hq, "H": r.H, "L": r.L, "S": r.S, "E": r.E,
                        "Ev": r.Ev, "mode": r.mode, "mask": r.mask_kind, "window": r.window,
                        "sink": r.sink != "none", "scale": r.scale,
                        "parallelism": f"replicas x{world} (independent batches, no collective)",
@@ -521,7 +556,8 @@ def reference(args):
         "metric": METRIC, "value": round(value, 6), "unit": smp.unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": r.name, "N": r.N, "Hq": r.Hq, "H": r.H, "L": r.L, "S": r.S, "E": r.E,
+        "config": {"workload": r.name, **({"keys_listed_per_kv_head": r.n_sel} if r.n_sel > 0 else {}),
+                   "N": r.N, "Hq": r.Hq, "H": r.H, "L": r.L, "S": r.S, "E": r.E,
                    "Ev": r.Ev, "mode": r.mode, "mask": r.mask_kind},
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 6), "unit": smp.unit, "cores": _oracle_cores(), "kind": "oracle",
@@ -541,12 +577,20 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch N (profiling captures of a smaller case)")
+    ap.add_argument("--select", type=int, default=None, metavar="K",
+                    help="decode workloads: attend over K listed keys per KV head (attn_decode_indexed), "
+                         "a random K-subset of the cache")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    import dataclasses
     if args.batch is not None:
-        import dataclasses
         sw.RECIPES[args.workload] = dataclasses.replace(sw.RECIPES[args.workload], N=args.batch)
+    if args.select is not None:
+        rr = sw.RECIPES[args.workload]
+        if args.select < 1 or not is_decode(rr):
+            raise SystemExit("--select needs K >= 1 and a decode-shaped bf16 workload")
+        sw.RECIPES[args.workload] = dataclasses.replace(rr, n_sel=args.select)
     if args.impl == "reference":
         reference(args)
     else:

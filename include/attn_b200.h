@@ -126,6 +126,41 @@ int attn_fwd_streaming(const void* q, const void* k, const void* v, void* out, f
                        const float* sink_logits, int window, int keep_first, const float* bias,
                        int dtype, void* stream);
 
+/*
+ * attn_decode_indexed -- exact decode attention over a listed subset of the
+ * cached keys: the step that follows a top-k key selection (page "기술 요약:
+ * SOCKET - 희소 어텐션을 위한 SOft Collision Kernel EsTimator", 방법론, 핵심
+ * 메커니즘 step 4: the top-k keys are chosen, then exact attention is computed
+ * on that subset).  The selection itself is the caller's.
+ *
+ *   key_idx  [N, H, n_sel] int32, device memory owned by the caller: the key
+ *            positions (rows of k and v) each (batch, KV head) attends to.  One
+ *            list serves all Hq/H query heads of the KV group and all L query
+ *            rows.  Entries outside [0, S) (such as -1 padding) select nothing.
+ *            A position listed twice counts twice (attention over the gathered
+ *            list).  Order does not matter.
+ *   n_sel    >= 1, entries per list.
+ *
+ * The softmax and the value sum run over the listed keys only:
+ *   out_i = sum_{j in list} e^{z_ij} v_j / (e^{s} [sink] + sum_{j in list} e^{z_ij})
+ * with z_ij = scale * <q_i, k_j>.  mask_kind (NONE, CAUSAL, SLIDING_WINDOW with
+ * window), bias [L, S] and the sink are those of attn_fwd, applied at each
+ * key's original position j.  A row that sees no listed key gets out = 0 and
+ * lse = -inf (lse = s with a sink).
+ *
+ * q, k, v, out, lse: attn_fwd's layouts, bf16 only (dot score).  The call must
+ * be decode-shaped, (Hq/H)*L <= 16, else ATTN_ERR_NOT_DECODE.  Errors: attn_fwd's
+ * codes, plus ATTN_ERR_NULL_POINTER for a NULL key_idx, ATTN_ERR_BAD_SHAPE for
+ * n_sel < 1, ATTN_ERR_ALIGNMENT for a key_idx not 4-byte aligned.  It uses and
+ * grows the same library workspace as attn_fwd's decode path (ordering rules
+ * as there) and returns without a host synchronisation.
+ */
+int attn_decode_indexed(const void* q, const void* k, const void* v, void* out, float* lse,
+                        const int* key_idx, int n_sel,
+                        int N, int Hq, int H, int L, int S, int E, int Ev, float scale,
+                        const float* sink_logits, int mask_kind, int window, const float* bias,
+                        void* stream);
+
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* attn_status_string(int status);
 

@@ -100,6 +100,8 @@ def generate_on_device(r: sw.Recipe, device="cuda") -> dict:
     out["sink"] = None if s is None else torch.from_numpy(s).to(device)
     b = sw.bias_matrix(r)
     out["bias"] = None if b is None else torch.from_numpy(b).to(device)
+    ki = sw.key_index_set(r)
+    out["key_idx"] = None if ki is None else torch.from_numpy(ki).to(device)
     return out
 
 

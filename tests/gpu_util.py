@@ -25,6 +25,11 @@ def api_mode(r: sw.Recipe) -> str:
 
 
 def run_gpu(r: sw.Recipe, t: dict):
+    if r.n_sel > 0:
+        out, lse = attn.attn_decode_indexed(t["q"], t["k"], t["v"], t["key_idx"], scale=r.scale, sink=t["sink"],
+                                            mask_kind=r.mask_kind, window=r.window, bias=t["bias"])
+        torch.cuda.synchronize()
+        return out, lse
     out, lse = attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=api_mode(r), sink=t["sink"],
                              mask_kind=r.mask_kind, window=r.window, bias=t["bias"], keep_first=r.keep)
     torch.cuda.synchronize()
@@ -39,6 +44,19 @@ def oracle_rows(r: sw.Recipe, n: int, hq: int, rows, host: dict | None = None):
     """Oracle out (R, Ev) and lse (R,) for query rows of (n, hq), from host-regenerated inputs."""
     rows = np.asarray(rows, dtype=np.int64)
     kvh = hq // r.group
+    if r.n_sel > 0:
+        # the index-set oracle on this query head alone (one KV head, all L rows), then the rows asked for
+        q = sw.tensor_slice_f64(r, "q", n, hq)[None, None]
+        k = sw.tensor_slice_f64(r, "k", n, kvh)[None, None]
+        v = sw.tensor_slice_f64(r, "v", n, kvh)[None, None]
+        idx = (host["key_idx"] if host is not None else sw.key_index_set(r))[n, kvh][None, None]
+        sink = sw.sink_logits(r)
+        bias = sw.bias_matrix(r)
+        o, l = orc.attention_over_index_set(q, k, v, idx, scale=r.scale,
+                                            sink=None if sink is None else sink[hq:hq + 1].astype(np.float64),
+                                            mask_kind=r.mask_kind, window=r.window,
+                                            bias=None if bias is None else bias.astype(np.float64))
+        return o[0, 0, rows], l[0, 0, rows]
     if host is not None:
         q = sw.as_f64(r, host["q"][n, hq])
         k = sw.as_f64(r, host["k"][n, kvh])
@@ -86,12 +104,21 @@ def small_recipe(name, **kw) -> sw.Recipe:
     return sw.Recipe(name, **base)
 
 
-def run_and_check_full(r: sw.Recipe):
-    """Whole-tensor comparison for small recipes."""
+def run_and_check_full(r: sw.Recipe, key_idx: np.ndarray | None = None):
+    """Whole-tensor comparison for small recipes (key_idx overrides the recipe's key lists)."""
     host = sw.generate(r)
     t = {k: sgpu.to_device(host[k], r) for k in ("q", "k", "v")}
     t["sink"] = None if host["sink"] is None else torch.from_numpy(host["sink"]).cuda()
     t["bias"] = None if host["bias"] is None else torch.from_numpy(host["bias"]).cuda()
+    if r.n_sel > 0:
+        idx = host["key_idx"] if key_idx is None else key_idx
+        t["key_idx"] = torch.from_numpy(np.ascontiguousarray(idx, dtype=np.int32)).cuda()
+        out, lse = run_gpu(r, t)
+        ref_out, ref_lse = orc.attention_over_index_set(
+            sw.as_f64(r, host["q"]), sw.as_f64(r, host["k"]), sw.as_f64(r, host["v"]), idx, scale=r.scale,
+            sink=None if host["sink"] is None else host["sink"].astype(np.float64), mask_kind=r.mask_kind,
+            window=r.window, bias=None if host["bias"] is None else host["bias"].astype(np.float64))
+        return compare(r, out_to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, r.name)
     out, lse = run_gpu(r, t)
     ref_out, ref_lse = orc.attention_forward(
         sw.as_f64(r, host["q"]), sw.as_f64(r, host["k"]), sw.as_f64(r, host["v"]), scale=r.scale, mode=r.mode,

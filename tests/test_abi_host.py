@@ -94,6 +94,26 @@ def test_streaming_argument_validation(lib, kw, status):
     assert call_streaming(**kw) == status
 
 
+def call_indexed(**kw):
+    a = dict(q=P, k=P, v=P, out=P, lse=P, idx=P, n_sel=8, N=1, Hq=2, H=1, L=1, S=64, E=64, Ev=64, scale=0.125,
+             sink=None, mask_kind=0, window=0, bias=None, stream=None)
+    a.update(kw)
+    return attn.attn_decode_indexed_raw(a["q"], a["k"], a["v"], a["out"], a["lse"], a["idx"], a["n_sel"], a["N"],
+                                        a["Hq"], a["H"], a["L"], a["S"], a["E"], a["Ev"], a["scale"], a["sink"],
+                                        a["mask_kind"], a["window"], a["bias"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(idx=None), -1), (dict(q=None), -1), (dict(n_sel=0), -2), (dict(n_sel=-4), -2),
+    (dict(N=0), -2), (dict(Hq=3, H=2), -3), (dict(E=96), -4), (dict(scale=0.0), -5),
+    (dict(mask_kind=3), -7), (dict(mask_kind=2, window=0), -8),
+    (dict(idx=P + 2), -11), (dict(v=P + 8), -11),
+    (dict(Hq=32, H=1), -17), (dict(Hq=4, H=1, L=5), -17),
+])
+def test_indexed_argument_validation(lib, kw, status):
+    assert call_indexed(**kw) == status
+
+
 def test_python_binding_rejects_cpu_tensors(lib):
     import torch
     q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)

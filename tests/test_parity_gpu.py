@@ -97,6 +97,42 @@ DECODE_CASES = [
 ]
 
 
+# exact decode over a listed key subset (a top-k selection's output)
+INDEXED_CASES = [
+    R("ix_L1_g4_S1000_sel100_sink", L=1, S=1000, E=128, Ev=128, N=2, Hq=8, H=2, n_sel=100, sink="normal",
+      scale=0.0884),
+    R("ix_L1_S5000_sel333_e64", L=1, S=5000, N=1, Hq=2, H=2, n_sel=333),
+    R("ix_L4_g4_S300_sel50_causal", L=4, S=300, Hq=8, H=2, n_sel=50, mask_kind="causal", sink="normal"),
+    R("ix_L2_g2_S300_sel90_window_bias", L=2, S=300, Hq=2, H=1, n_sel=90, mask_kind="window", window=50,
+      bias="random10"),
+    R("ix_sel1", L=1, S=200, Hq=4, H=4, n_sel=1),
+    R("ix_sel_over_S_repeats", L=1, S=50, Hq=2, H=1, n_sel=130, sink="normal"),
+    R("ix_many_units", L=1, S=2000, N=40, Hq=16, H=8, E=128, Ev=128, n_sel=70, scale=0.0884),
+    R("ix_e64_ev128_g16", L=1, S=700, Hq=16, H=1, E=64, Ev=128, n_sel=200),
+    R("ix_e128_ev64_L3_g5", L=3, S=400, Hq=5, H=1, E=128, Ev=64, n_sel=129, mask_kind="causal"),
+]
+
+
+@pytest.mark.parametrize("r", INDEXED_CASES, ids=lambda r: r.name)
+def test_decode_indexed_small(r):
+    gu.run_and_check_full(r)
+
+
+def test_decode_indexed_padding_and_duplicates():
+    """-1 and >= S entries select nothing; a listed duplicate counts twice; an all-padding list gives
+    out = 0 and lse = -inf (lse = sink with a sink)."""
+    r = R("ix_pad", L=2, S=300, Hq=4, H=2, n_sel=40, sink="normal")
+    idx = sw.key_index_set(r).copy()
+    idx[0, 0, :5] = -1
+    idx[0, 1, 7] = 300
+    idx[1 % r.N, 1, 9] = 10**6
+    idx[0, 0, 20] = idx[0, 0, 21]
+    gu.run_and_check_full(r, idx)
+    for sink in ("none", "normal"):
+        r0 = R("ix_all_pad", L=1, S=100, Hq=2, H=2, n_sel=70, sink=sink)
+        gu.run_and_check_full(r0, np.full((r0.N, r0.H, 70), -1, dtype=np.int32))
+
+
 @pytest.mark.parametrize("r", PREFILL_CASES, ids=lambda r: r.name)
 def test_prefill_bf16_small(r):
     gu.run_and_check_full(r)
@@ -152,6 +188,23 @@ def test_repeat_calls_are_deterministic():
 
 FULL = ["dot_causal_2k_bf16", "dot_bias10_2k_f32", "rbf_registers_4k_bf16", "sink_gqa_window_16k_bf16",
         "decode_sink_gqa_128k_bf16"]
+
+
+def test_decode_indexed_full_size_top_k_33x():
+    """The long-context decode workload (N=32, 32 query / 8 KV heads, S=131072, E=128) over a
+    33x-sparse selection (3972 keys per KV head), sampled units against the oracle."""
+    import dataclasses
+    r = dataclasses.replace(sw.RECIPES["decode_sink_gqa_128k_bf16"], name="decode_top_k_33x", n_sel=3972)
+    t = sgpu.generate_on_device(r)
+    out, lse = gu.run_gpu(r, t)
+    assert torch.isfinite(out.float()).all()
+    host = {"key_idx": sw.key_index_set(r)}
+    for n, hq in ((0, 0), (r.N - 1, r.Hq - 1), (17, 13)):
+        ref_out, ref_lse = gu.oracle_rows(r, n, hq, [0], host)
+        gu.compare(r, gu.out_to_f64(out[n, hq, [0]]), lse[n, hq, [0]].cpu().numpy(), ref_out, ref_lse,
+                   f"top-k n={n} hq={hq}")
+    del t, out, lse
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("name", FULL)

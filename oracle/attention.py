@@ -34,6 +34,12 @@ in blocks of query rows so that memory stays bounded:
   out = sum_{j in A} e^{z_j-M} v_j / D,  lse = M + ln D.
 * A row with no visible key and no sink gives out = 0 and lse = -inf (page
   "SDPA란 무엇인가" §4: SDPA returns 0 instead of NaN for a fully masked row).
+* Boolean keep mask and key padding (page "SDPA란 무엇인가" §1: B is 0 or
+  -inf; §4 trap 1: a boolean attn_mask marks with True the pairs that take
+  part, the opposite of key_padding_mask; the left-padding check: with the
+  mask passed, padded and unpadded inputs give the same output for the real
+  tokens): key j is visible to row i only where keep[i, j] is True and, for
+  batch n, kv_start[n] <= j < kv_end[n].  Both compose with every mask kind.
 * Exact attention over a selected key subset (page "기술 요약: SOCKET - 희소
   어텐션을 위한 SOft Collision Kernel EsTimator", 방법론, 핵심 메커니즘 step 4:
   the top-k keys are picked, then exact attention runs on that subset): the
@@ -115,12 +121,23 @@ def softmax_with_sink(z: np.ndarray, vis: np.ndarray, sink: float | None):
     return alpha, p_sink, lse
 
 
+def padded_visible(vis: np.ndarray, keep_rows=None, kv_range=None) -> np.ndarray:
+    """Narrow a visibility matrix (R, S) by a boolean keep matrix (R, S) and a key range (start, end)."""
+    if keep_rows is not None:
+        vis = vis & np.asarray(keep_rows, dtype=bool)
+    if kv_range is not None:
+        j = np.arange(vis.shape[1])[None, :]
+        vis = vis & (j >= kv_range[0]) & (j < kv_range[1])
+    return vis
+
+
 def attend_rows(q_rows, rows, k, v, L, *, scale, mode="dot", sink=None, mask_kind="none",
-                window=0, bias_rows=None, return_weights=False, keep=0):
+                window=0, bias_rows=None, return_weights=False, keep=0, keep_rows=None, kv_range=None):
     """Attention of query rows ``q_rows`` (R, E) at positions ``rows`` against one KV head.
 
-    k (S, E), v (S, Ev), bias_rows (R, S) or None.  Returns out (R, Ev) and
-    lse (R,) (and the weights and sink probability when asked).
+    k (S, E), v (S, Ev), bias_rows (R, S) or None, keep_rows (R, S) bool or
+    None, kv_range (start, end) or None.  Returns out (R, Ev) and lse (R,)
+    (and the weights and sink probability when asked).
     """
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -128,7 +145,7 @@ def attend_rows(q_rows, rows, k, v, L, *, scale, mode="dot", sink=None, mask_kin
     z = logits(q_rows, k, scale, mode)
     if bias_rows is not None:
         z = z + np.asarray(bias_rows, dtype=np.float64)
-    vis = visible(rows, S, L, mask_kind, window, keep)
+    vis = padded_visible(visible(rows, S, L, mask_kind, window, keep), keep_rows, kv_range)
     alpha, p_sink, lse = softmax_with_sink(z, vis, sink)
     out = alpha @ v
     if return_weights:
@@ -137,11 +154,12 @@ def attend_rows(q_rows, rows, k, v, L, *, scale, mode="dot", sink=None, mask_kin
 
 
 def attention_forward(q, k, v, *, scale, mode="dot", sink=None, mask_kind="none", window=0,
-                      bias=None, row_block=128, keep=0):
+                      bias=None, row_block=128, keep=0, mask_keep=None, kv_start=None, kv_end=None):
     """Whole forward: q (N,Hq,L,E), k (N,H,S,E), v (N,H,S,Ev) float64.
 
     sink: per-query-head logits (Hq,) or None.  bias: (L, S) or None.
-    Returns out (N,Hq,L,Ev) and lse (N,Hq,L).
+    mask_keep: (L, S) bool or None.  kv_start, kv_end: (N,) ints or None
+    (0 and S).  Returns out (N,Hq,L,Ev) and lse (N,Hq,L).
     """
     q = np.asarray(q, dtype=np.float64)
     N, Hq, L, _ = q.shape
@@ -159,9 +177,14 @@ def attention_forward(q, k, v, *, scale, mode="dot", sink=None, mask_kind="none"
             for i0 in range(0, L, row_block):
                 rows = np.arange(i0, min(L, i0 + row_block))
                 b = None if bias is None else np.asarray(bias)[rows]
+                kr = None if mask_keep is None else np.asarray(mask_keep, dtype=bool)[rows]
+                rng = None
+                if kv_start is not None or kv_end is not None:
+                    rng = (0 if kv_start is None else int(kv_start[n]),
+                           k.shape[2] if kv_end is None else int(kv_end[n]))
                 o, l = attend_rows(q[n, hq, rows], rows, k[n, kvh], v[n, kvh], L, scale=scale,
                                    mode=mode, sink=s, mask_kind=mask_kind, window=window,
-                                   bias_rows=b, keep=keep)
+                                   bias_rows=b, keep=keep, keep_rows=kr, kv_range=rng)
                 out[n, hq, rows] = o
                 lse[n, hq, rows] = l
     return out, lse

@@ -102,6 +102,11 @@ def generate_on_device(r: sw.Recipe, device="cuda") -> dict:
     out["bias"] = None if b is None else torch.from_numpy(b).to(device)
     ki = sw.key_index_set(r)
     out["key_idx"] = None if ki is None else torch.from_numpy(ki).to(device)
+    km = sw.keep_matrix(r)
+    out["mask_bits"] = None if km is None else torch.from_numpy(sw.pack_mask_bits(km).view(np.int32)).to(device)
+    ks, ke = sw.kv_ranges(r)
+    out["kv_start"] = None if ks is None else torch.from_numpy(ks).to(device)
+    out["kv_end"] = None if ke is None else torch.from_numpy(ke).to(device)
     return out
 
 

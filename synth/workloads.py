@@ -49,6 +49,7 @@ STREAM_SINK = 4
 STREAM_BIAS = 5
 STREAM_KEY_FACTOR = 6
 STREAM_KEY_INDEX = 7
+STREAM_PAD = 8
 
 LN2 = 0.6931471805599453          # double nearest ln 2
 HALF_PI = 1.5707963267948966      # double nearest pi/2
@@ -227,6 +228,9 @@ class Recipe:
     window: int = 0
     keep: int = 0         # streaming mask: initial tokens every later query sees
     n_sel: int = 0        # > 0: decode over a selected key list of this length per (n, KV head)
+    keep_mask: str = "none"   # "random10": boolean keep mask, False where the random10 bias is -inf
+    pad_left: float = 0.0     # per-batch left padding: kv_start[n] = floor(u * pad_left * S)
+    pad_right: float = 0.0    # per-batch right padding: kv_end[n] = S - floor(u * pad_right * S)
     sink: str = "none"    # "none", "fixed", "normal"
     sink_values: tuple = ()
     bias: str = "none"    # "none" or "random10"
@@ -340,6 +344,40 @@ def bias_matrix(r: Recipe):
     return b.astype(np.float32)
 
 
+def keep_matrix(r: Recipe) -> np.ndarray | None:
+    """(L, S) bool keep mask or None.  random10: the complement of the random10
+    bias pattern (the same draws): False with probability 0.1, True on the
+    diagonal j == i."""
+    if r.keep_mask == "none":
+        return None
+    u = uniform_f64(stream_key(r.seed, STREAM_BIAS), 0, r.L * r.S).reshape(r.L, r.S)
+    keep = u >= 0.1
+    idx = np.arange(min(r.L, r.S))
+    keep[idx, idx] = True
+    return keep
+
+
+def pack_mask_bits(keep: np.ndarray) -> np.ndarray:
+    """(L, S) bool -> (L, ceil(S/32)) uint32: bit j % 32 of word j // 32 is keep[:, j]
+    (bits past S are 0)."""
+    keep = np.asarray(keep, dtype=bool)
+    L, S = keep.shape
+    W = (S + 31) // 32
+    padded = np.zeros((L, W * 32), dtype=bool)
+    padded[:, :S] = keep
+    return np.packbits(padded.reshape(L, W, 4, 8), axis=-1, bitorder="little").reshape(L, W * 4).view("<u4").copy()
+
+
+def kv_ranges(r: Recipe):
+    """(kv_start, kv_end) int32 arrays of length N, or (None, None) without padding."""
+    if r.pad_left <= 0 and r.pad_right <= 0:
+        return None, None
+    u = uniform_f64(stream_key(r.seed, STREAM_PAD), 0, 2 * r.N).reshape(2, r.N)
+    start = np.floor(u[0] * r.pad_left * r.S).astype(np.int32)
+    end = (r.S - np.floor(u[1] * r.pad_right * r.S)).astype(np.int32)
+    return start, end
+
+
 def key_index_set(r: Recipe) -> np.ndarray | None:
     """(N, H, n_sel) int32 key lists, or None.  For each (n, KV head) one uniform
     draw per cached key; the n_sel keys with the largest draws, in decreasing
@@ -371,6 +409,8 @@ def generate(r: Recipe) -> dict:
     out["sink"] = sink_logits(r)
     out["bias"] = bias_matrix(r)
     out["key_idx"] = key_index_set(r)
+    out["keep"] = keep_matrix(r)
+    out["kv_start"], out["kv_end"] = kv_ranges(r)
     return out
 
 

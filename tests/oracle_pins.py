@@ -436,10 +436,58 @@ def check_index_set(seed=15):
             assert np.allclose(l[n, hq], z, atol=1e-13)
 
 
+def check_padding_and_keep_mask(seed=16):
+    """Keep mask and key padding: a keep mask equals the 0/-inf bias; key ranges
+    equal the keep mask built from them; a left-padded input with kv_start = pad
+    gives the unpadded input's output on the real tokens (the page's left-padding
+    check), whatever the padding holds; left-padded start rows under a causal mask
+    see no key (out 0, lse -inf; with a sink lse = s); kv_end = m equals keys and
+    values cut to m."""
+    rng = np.random.default_rng(seed)
+    N, H, Hq, E, Ev = 2, 2, 4, 6, 5
+    sink = rng.standard_normal(Hq)
+    # keep mask == additive 0/-inf bias
+    L, S = 7, 23
+    q, k, v = _rand(rng, N, Hq, L, E), _rand(rng, N, H, S, E), _rand(rng, N, H, S, Ev)
+    keep = rng.random((L, S)) < 0.6
+    for mk in ("none", "causal"):
+        a = orc.attention_forward(q, k, v, scale=0.4, sink=sink, mask_kind=mk, mask_keep=keep)
+        b = orc.attention_forward(q, k, v, scale=0.4, sink=sink, mask_kind=mk, bias=np.where(keep, 0.0, -np.inf))
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1]), mk
+    # key ranges == the keep mask of the same range (per batch)
+    ks, ke = np.array([3, 0]), np.array([19, 11])
+    r1 = orc.attention_forward(q, k, v, scale=0.4, sink=sink, kv_start=ks, kv_end=ke)
+    for n in range(N):
+        km = np.zeros((L, S), dtype=bool)
+        km[:, ks[n]:ke[n]] = True
+        r2 = orc.attention_forward(q[n:n + 1], k[n:n + 1], v[n:n + 1], scale=0.4, sink=sink, mask_keep=km)
+        assert np.array_equal(r1[0][n:n + 1], r2[0]) and np.array_equal(r1[1][n:n + 1], r2[1])
+    # left padding: the real tokens' outputs do not depend on the padding
+    L0, P = 9, 5
+    q0, k0, v0 = _rand(rng, N, Hq, L0, E), _rand(rng, N, H, L0, E), _rand(rng, N, H, L0, Ev)
+    pad = lambda x: np.concatenate([100.0 * _rand(rng, *x.shape[:2], P, x.shape[3]), x], axis=2)  # noqa: E731
+    qp, kp, vp = pad(q0), pad(k0), pad(v0)
+    for mk in ("none", "causal"):
+        ref = orc.attention_forward(q0, k0, v0, scale=0.4, sink=sink, mask_kind=mk)
+        got = orc.attention_forward(qp, kp, vp, scale=0.4, sink=sink, mask_kind=mk, kv_start=np.full(N, P))
+        assert np.allclose(got[0][:, :, P:], ref[0], atol=1e-13) and np.allclose(got[1][:, :, P:], ref[1], atol=1e-13)
+        if mk == "causal":
+            # start rows see only padding
+            nos = orc.attention_forward(qp, kp, vp, scale=0.4, mask_kind=mk, kv_start=np.full(N, P))
+            assert np.all(nos[0][:, :, :P] == 0.0) and np.all(nos[1][:, :, :P] == -np.inf)
+            assert np.all(got[0][:, :, :P] == 0.0)
+            assert np.allclose(got[1][:, :, :P], np.broadcast_to(sink[None, :, None], (N, Hq, P)))
+    # right padding: kv_end = m equals cutting K and V to m keys (no position-dependent mask)
+    m = 15
+    cut = orc.attention_forward(q, k[:, :, :m], v[:, :, :m], scale=0.4, sink=sink)
+    end = orc.attention_forward(q, k, v, scale=0.4, sink=sink, kv_end=np.full(N, m))
+    assert np.allclose(end[0], cut[0], atol=1e-13) and np.allclose(end[1], cut[1], atol=1e-13)
+
+
 ALL_CHECKS = [
     check_dot_matches_sdpa, check_brute_force, check_rbf_expansion, check_rbf_limits,
     check_dot_limits, check_uniform_entropy_golden, check_sink_limit, check_sink_mass,
     check_zero_sink_equivalence, check_convexity, check_causal_alignment_golden,
     check_fully_masked_rows, check_window_semantics, check_permutation_equivariance,
-    check_gqa_repeat, check_streaming_mask, check_index_set,
+    check_gqa_repeat, check_streaming_mask, check_index_set, check_padding_and_keep_mask,
 ]

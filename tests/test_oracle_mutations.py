@@ -84,7 +84,27 @@ def _select_ignored(sel, S):
     return np.arange(S)  # attends over the whole cache
 
 
+_real_padded_visible = orc.padded_visible
+
+
+def _padding_range_ignored(vis, keep_rows=None, kv_range=None):
+    return _real_padded_visible(vis, keep_rows, None)
+
+
+def _keep_mask_inverted(vis, keep_rows=None, kv_range=None):
+    inv = None if keep_rows is None else ~np.asarray(keep_rows, dtype=bool)
+    return _real_padded_visible(vis, inv, kv_range)
+
+
+def _padding_end_inclusive(vis, keep_rows=None, kv_range=None):
+    wide = None if kv_range is None else (kv_range[0], kv_range[1] + 1)
+    return _real_padded_visible(vis, keep_rows, wide)
+
+
 MUTATIONS = [
+    ("padded_visible", _padding_range_ignored, pins.check_padding_and_keep_mask),
+    ("padded_visible", _keep_mask_inverted, pins.check_padding_and_keep_mask),
+    ("padded_visible", _padding_end_inclusive, pins.check_padding_and_keep_mask),
     ("select_keys", _select_unique, pins.check_index_set),
     ("select_keys", _select_clipped, pins.check_index_set),
     ("select_keys", _select_ignored, pins.check_index_set),

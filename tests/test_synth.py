@@ -127,3 +127,28 @@ def test_key_index_set_is_a_random_subset():
     assert np.array_equal(big[0, 0, :10], big[0, 0, 10:20])
     assert sorted(big[0, 0, :10].tolist()) == list(range(10))
     assert sw.key_index_set(base) is None
+
+
+def test_pack_mask_bits_layout():
+    """Bit j % 32 of word j // 32 of row i is keep[i, j]; bits past S are zero."""
+    rng = np.random.default_rng(3)
+    for L, S in ((3, 1), (4, 31), (2, 32), (5, 77), (1, 128)):
+        keep = rng.random((L, S)) < 0.5
+        w = sw.pack_mask_bits(keep)
+        assert w.dtype == np.uint32 and w.shape == (L, (S + 31) // 32)
+        for i in range(L):
+            for j in range((S + 31) // 32 * 32):
+                bit = (int(w[i, j // 32]) >> (j % 32)) & 1
+                assert bit == (int(keep[i, j]) if j < S else 0), (L, S, i, j)
+
+
+def test_keep_matrix_matches_random10_bias_and_padding_ranges():
+    import dataclasses
+    base = sw.RECIPES["tiny_rbf_sink_causal_f32"]
+    r = dataclasses.replace(base, bias="random10", keep_mask="random10", L=50, S=70)
+    keep, bias = sw.keep_matrix(r), sw.bias_matrix(r)
+    assert np.array_equal(keep, bias == 0.0)
+    p = dataclasses.replace(base, N=64, S=1000, pad_left=0.25, pad_right=0.1)
+    ks, ke = sw.kv_ranges(p)
+    assert ks.min() >= 0 and ks.max() < 250 and ke.min() > 900 and ke.max() <= 1000 and len(set(ks)) > 10
+    assert sw.kv_ranges(base) == (None, None)

@@ -51,6 +51,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_decode_indexed.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, ci, cf, vp, ci, ci, vp,
                                         vp]
     lib.attn_decode_indexed.restype = ci
+    lib.attn_fwd_padded.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp, vp, vp, ci,
+                                    vp]
+    lib.attn_fwd_padded.restype = ci
     lib.attn_status_string.argtypes = [ci]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_release_workspace.argtypes = []
@@ -92,6 +95,16 @@ def attn_fwd_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H, L, S, E, Ev, s
                         int(window), c(bias_ptr), int(dtype), c(stream_ptr))
 
 
+def attn_fwd_padded_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H, L, S, E, Ev, scale, mode, sink_ptr,
+                        mask_kind, window, bits_ptr, start_ptr, end_ptr, dtype, stream_ptr) -> int:
+    """The keep-bits / key-padding C entry point with integer pointers; returns the status code."""
+    lib = load_library()
+    c = lambda p: None if p is None else ctypes.c_void_p(int(p))  # noqa: E731
+    return lib.attn_fwd_padded(c(q_ptr), c(k_ptr), c(v_ptr), c(out_ptr), c(lse_ptr), int(N), int(Hq), int(H), int(L),
+                               int(S), int(E), int(Ev), float(scale), int(mode), c(sink_ptr), int(mask_kind),
+                               int(window), c(bits_ptr), c(start_ptr), c(end_ptr), int(dtype), c(stream_ptr))
+
+
 def attn_fwd_streaming_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H, L, S, E, Ev, scale, mode, sink_ptr,
                            window, keep_first, bias_ptr, dtype, stream_ptr) -> int:
     """The streaming-mask C entry point with integer pointers; returns the status code."""
@@ -105,7 +118,9 @@ def attn_fwd_streaming_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H, L, S
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float, mode: str = "dot",
              sink: torch.Tensor | None = None, mask_kind: str = "none", window: int = 0,
              bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
-             lse: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None, keep_first: int = 0):
+             lse: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None, keep_first: int = 0,
+             mask_bits: torch.Tensor | None = None, kv_start: torch.Tensor | None = None,
+             kv_end: torch.Tensor | None = None):
     """out = softmax(z + B) V on the GPU.  Returns (out, lse).
 
     q (N, Hq, L, E), k (N, H, S, E), v (N, H, S, Ev): contiguous CUDA tensors,
@@ -113,7 +128,9 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float,
     float32 or None.  mode: "dot", "rbf" or "sink"; mask_kind: "none",
     "causal", "window" or "streaming" (the first ``keep_first`` keys plus the
     last ``window`` keys, through attn_fwd_streaming).  out/lse may be given
-    (contiguous, right shape).
+    (contiguous, right shape).  mask_bits (L, ceil(S/32)) int32 (bit j%32 of
+    word j/32 set: row may attend key j), kv_start / kv_end (N,) int32 key
+    padding: any of them routes the call through attn_fwd_padded (no bias).
     """
     if mask_kind not in MASKS and mask_kind != "streaming":
         raise ValueError(f"unknown mask kind {mask_kind!r}")
@@ -151,7 +168,19 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float,
         common = (_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), N, Hq, H, L, S, E, Ev, float(scale), MODES[mode],
                   _ptr(sink))
         tail = (_ptr(bias), DTYPES[q.dtype], ctypes.c_void_p(stream.cuda_stream))
-        if mask_kind == "streaming":
+        padded = mask_bits is not None or kv_start is not None or kv_end is not None
+        if padded:
+            if bias is not None or mask_kind == "streaming":
+                raise ValueError("mask_bits / kv_start / kv_end combine with none, causal or window masks only, "
+                                 "without a bias")
+            for name, t, shape in (("mask_bits", mask_bits, (L, (S + 31) // 32)), ("kv_start", kv_start, (N,)),
+                                   ("kv_end", kv_end, (N,))):
+                if t is not None and (not t.is_cuda or t.dtype != torch.int32 or tuple(t.shape) != shape
+                                      or not t.is_contiguous()):
+                    raise ValueError(f"{name} must be a contiguous CUDA int32 tensor of shape {shape}")
+            st = lib.attn_fwd_padded(*common, MASKS[mask_kind], int(window), _ptr(mask_bits), _ptr(kv_start),
+                                     _ptr(kv_end), *tail[1:])
+        elif mask_kind == "streaming":
             st = lib.attn_fwd_streaming(*common, int(window), int(keep_first), *tail)
         else:
             st = lib.attn_fwd(*common, MASKS[mask_kind], int(window), *tail)

@@ -127,8 +127,12 @@ int validate(const void* q, const void* k, const void* v, void* out, float* lse,
 
 AttnArgs make_args(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L,
                    int S, int E, int Ev, float scale, int mode, const float* sink_logits, int mask_kind, int window,
-                   int keep, const float* bias) {
+                   int keep, const float* bias, const uint32_t* mask_bits = nullptr, const int* kv_start = nullptr,
+                   const int* kv_end = nullptr) {
   AttnArgs a{};
+  a.mask_bits = mask_bits;
+  a.kv_start = kv_start;
+  a.kv_end = kv_end;
   a.q = q;
   a.k = k;
   a.v = v;
@@ -155,14 +159,15 @@ AttnArgs make_args(const void* q, const void* k, const void* v, void* out, float
 // validates the rest and dispatches (fp32 kernel, split-key decode, tcgen05 prefill).
 int forward(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L, int S,
             int E, int Ev, float scale, int mode, const float* sink_logits, int mask_kind, int window, int keep,
-            const float* bias, int dtype, void* stream_ptr) {
+            const float* bias, int dtype, void* stream_ptr, const uint32_t* mask_bits = nullptr,
+            const int* kv_start = nullptr, const int* kv_end = nullptr) {
   const int st = validate(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, bias, dtype);
   if (st != ATTN_OK) return st;
   int dev = 0, sms = 0, major = 0;
   if (device_info(&dev, &sms, &major) != ATTN_OK) return ATTN_ERR_CUDA;
   if (major != 10) return ATTN_ERR_DEVICE;
-  const AttnArgs a =
-      make_args(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, mask_kind, window, keep, bias);
+  const AttnArgs a = make_args(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, mask_kind, window,
+                               keep, bias, mask_bits, kv_start, kv_end);
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
 
   if (dtype == ATTN_FP32) return launch_fp32(a, stream);
@@ -196,6 +201,19 @@ int attn_fwd_streaming(const void* q, const void* k, const void* v, void* out, f
   if (keep_first < 0) return ATTN_ERR_KEEP;
   return attn::forward(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, attn::MASK_STREAM,
                        window, keep_first, bias, dtype, stream_ptr);
+}
+
+int attn_fwd_padded(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L,
+                    int S, int E, int Ev, float scale, int mode, const float* sink_logits, int mask_kind, int window,
+                    const unsigned int* mask_bits, const int* kv_start, const int* kv_end, int dtype,
+                    void* stream_ptr) {
+  using namespace attn;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_SLIDING_WINDOW) return ATTN_ERR_MASK;
+  if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window < 1) return ATTN_ERR_WINDOW;
+  if ((mask_bits && !aligned(mask_bits, 4)) || (kv_start && !aligned(kv_start, 4)) || (kv_end && !aligned(kv_end, 4)))
+    return ATTN_ERR_ALIGNMENT;
+  return forward(q, k, v, out, lse, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, mask_kind, window, 0, nullptr,
+                 dtype, stream_ptr, mask_bits, kv_start, kv_end);
 }
 
 int attn_decode_indexed(const void* q, const void* k, const void* v, void* out, float* lse, const int* key_idx,

@@ -73,13 +73,17 @@ struct DecodeParams {  // 128 bytes: kept at that size, the kernels' code genera
 };
 static_assert(sizeof(DecodeParams) == 128, "DecodeParams layout");
 
-// GATHER only: the key lists and the K/V base pointers (a separate kernel argument,
-// so the other variants' parameter block stays as it is)
-struct GatherArgs {
-  const int* idx;            // [N*H][n_sel] key positions
-  const __nv_bfloat16* k;    // [N*H][S][E]
-  const __nv_bfloat16* v;    // [N*H][S][Ev]
+// GATHER and EXT only (a separate kernel argument, so the other variants'
+// parameter block stays as it is)
+struct ExtraArgs {
+  const int* idx;            // GATHER: [N*H][n_sel] key positions
+  const __nv_bfloat16* k;    // GATHER: [N*H][S][E]
+  const __nv_bfloat16* v;    // GATHER: [N*H][S][Ev]
   int n_sel;
+  const uint32_t* bits;      // EXT: [L][words] keep bits (bit j % 32 of word j / 32), or nullptr
+  const int* kv_start;       // EXT: [N] first non-padding key, or nullptr
+  const int* kv_end;         // EXT: [N] one past the last non-padding key, or nullptr
+  int words;                 // EXT: ceil(S / 32)
 };
 
 template <int E, int EV, bool GATHER = false>
@@ -144,10 +148,10 @@ __device__ __forceinline__ uint32_t sw_off(int row, int c16) {
   return (c16 >> 3) * (DC * 128) + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
 }
 
-template <int E, int EV, bool STREAM, bool GATHER>
+template <int E, int EV, bool STREAM, bool GATHER, bool EXT>
 __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
     decode_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                          const DecodeParams p, const GatherArgs ga) {
+                          const DecodeParams p, const ExtraArgs ga) {
   using C = DCfg<E, EV, GATHER>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -274,13 +278,15 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
   const int rA = lane >> 2;       // fragment rows rA and rA + 8
   const int cq = (lane & 3) * 2;  // fragment column pair
   const int off = p.S - p.L;
-  int lo_r[2], hi_r[2];
+  int lo_r[2], hi_r[2], row_i[2];
   bool live_r[2];
+  int ks_u = 0, ke_u = p.S;  // EXT: the current unit's non-padding keys
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int r = rA + 8 * h;
     live_r[h] = r < p.R;
     const int i = live_r[h] ? (r % p.L) : 0;
+    row_i[h] = i;
     lo_r[h] = (STREAM || p.mask_kind == MASK_WINDOW) ? i + off - p.window + 1 : 0;
     hi_r[h] = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, i + off + 1);
   }
@@ -374,6 +380,11 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
       cur_unit = u;
       load_q(u);
       reset_state();
+      if constexpr (EXT) {
+        const int n = static_cast<int>(u / p.H);
+        ks_u = ga.kv_start ? __ldg(ga.kv_start + n) : 0;
+        ke_u = ga.kv_end ? __ldg(ga.kv_end + n) : p.S;
+      }
     }
     const int idx = static_cast<int>(c - c_begin);
     const int s = idx % C::NSTAGE;
@@ -403,7 +414,7 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
       }
     }
     // logits in base 2, masks and bias
-    const bool need_mask = GATHER || p.mask_kind != MASK_NONE || p.bias != nullptr || key0 + 16 > p.S;
+    const bool need_mask = GATHER || EXT || p.mask_kind != MASK_NONE || p.bias != nullptr || key0 + 16 > p.S;
 #pragma unroll
     for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -418,6 +429,12 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
             if (key >= hi_r[h] || (key < lo_r[h] && key >= p.keep)) zz = -INFINITY;
           } else {
             if (key < lo_r[h] || key >= hi_r[h]) zz = -INFINITY;
+          }
+          if constexpr (EXT) {
+            if (key < ks_u || key >= ke_u) zz = -INFINITY;
+            if (ga.bits != nullptr && key < p.S &&
+                !((__ldg(ga.bits + static_cast<size_t>(row_i[h]) * ga.words + (key >> 5)) >> (key & 31)) & 1u))
+              zz = -INFINITY;
           }
           if (p.bias != nullptr && live_r[h] && key >= 0 && key < p.S)
             zz = fmaf(p.bias[static_cast<size_t>((rA + 8 * h) % p.L) * p.S + key], LOG2E, zz);
@@ -564,8 +581,8 @@ DecodePlan plan(const AttnArgs& a, int num_sms) {
   return d;
 }
 
-template <int E, int EV, bool STREAM, bool GATHER>
-int launch_decode_impl(const AttnArgs& a, const GatherArgs& ga, void* ws, size_t ws_bytes, int num_sms,
+template <int E, int EV, bool STREAM, bool GATHER, bool EXT>
+int launch_decode_impl(const AttnArgs& a, const ExtraArgs& ga, void* ws, size_t ws_bytes, int num_sms,
                        cudaStream_t stream) {
   using C = DCfg<E, EV, GATHER>;
   const DecodePlan d = GATHER ? plan_gather(a, ga.n_sel, num_sms) : plan(a, num_sms);
@@ -603,7 +620,7 @@ int launch_decode_impl(const AttnArgs& a, const GatherArgs& ga, void* ws, size_t
   p.G = d.G;
   p.max_segs = d.max_segs;
   p.c_dot = a.scale * LOG2E;
-  auto kern = decode_partial_kernel<E, EV, STREAM, GATHER>;
+  auto kern = decode_partial_kernel<E, EV, STREAM, GATHER, EXT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return -13;
   kern<<<d.G, GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, C::SMEM_BYTES, stream>>>(tk, tv, p, ga);
@@ -630,13 +647,13 @@ size_t decode_gather_workspace_bytes(const AttnArgs& a, int n_sel, int num_sms) 
 
 int launch_decode_gather_bf16(const AttnArgs& a, const int* key_idx, int n_sel, void* ws, size_t ws_bytes,
                               int num_sms, cudaStream_t stream) {
-  GatherArgs ga{};
+  ExtraArgs ga{};
   ga.idx = key_idx;
   ga.k = static_cast<const __nv_bfloat16*>(a.k);
   ga.v = static_cast<const __nv_bfloat16*>(a.v);
   ga.n_sel = n_sel;
 #define ATTN_GATHER_CASE(e, ev) \
-  if (a.E == e && a.Ev == ev) return launch_decode_impl<e, ev, false, true>(a, ga, ws, ws_bytes, num_sms, stream);
+  if (a.E == e && a.Ev == ev) return launch_decode_impl<e, ev, false, true, false>(a, ga, ws, ws_bytes, num_sms, stream);
   ATTN_GATHER_CASE(128, 128)
   ATTN_GATHER_CASE(64, 64)
   ATTN_GATHER_CASE(64, 128)
@@ -649,11 +666,18 @@ int launch_decode_bf16(const AttnArgs& a, void* ws, size_t ws_bytes, int num_sms
   // kept initial keys need the streaming mask test even where the plan makes no
   // head/window split (kept keys and window overlap: nc_head is then 0)
   const bool st = a.mask_kind == MASK_STREAM && a.keep > 0;
-  const GatherArgs none{};
-#define ATTN_DECODE_CASE(e, ev)                                                                          \
-  if (a.E == e && a.Ev == ev)                                                                            \
-    return st ? launch_decode_impl<e, ev, true, false>(a, none, ws, ws_bytes, num_sms, stream)           \
-              : launch_decode_impl<e, ev, false, false>(a, none, ws, ws_bytes, num_sms, stream);
+  const bool ext = a.mask_bits != nullptr || a.kv_start != nullptr || a.kv_end != nullptr;
+  ExtraArgs xa{};
+  xa.bits = a.mask_bits;
+  xa.kv_start = a.kv_start;
+  xa.kv_end = a.kv_end;
+  xa.words = (a.S + 31) / 32;
+#define ATTN_DECODE_CASE(e, ev)                                                                              \
+  if (a.E == e && a.Ev == ev) {                                                                              \
+    if (st) return launch_decode_impl<e, ev, true, false, false>(a, xa, ws, ws_bytes, num_sms, stream);    \
+    if (ext) return launch_decode_impl<e, ev, false, false, true>(a, xa, ws, ws_bytes, num_sms, stream);   \
+    return launch_decode_impl<e, ev, false, false, false>(a, xa, ws, ws_bytes, num_sms, stream);           \
+  }
   ATTN_DECODE_CASE(128, 128)
   ATTN_DECODE_CASE(64, 64)
   ATTN_DECODE_CASE(64, 128)

@@ -36,6 +36,10 @@ struct F32Params {
   int N, Hq, H, L, S, group;
   int mask_kind, window, keep;
   float scale;
+  const uint32_t* mask_bits;  // [L][mask_words] keep bits or nullptr
+  const int* kv_start;        // [N] or nullptr
+  const int* kv_end;          // [N] or nullptr
+  int mask_words;
 };
 
 template <int E, int EV>
@@ -84,8 +88,11 @@ __global__ void __launch_bounds__(FTHREADS) fp32_attn_kernel(const F32Params p) 
   const bool windowed = p.mask_kind == MASK_WINDOW || p.mask_kind == MASK_STREAM;
   const int hi_blk = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, r_last + off + 1);
   const int lo_blk = (windowed && p.keep == 0) ? max(0, r0 + off - p.window + 1) : 0;
-  const int jb_lo = lo_blk / FBN;
-  const int jb_hi = hi_blk > lo_blk ? (hi_blk + FBN - 1) / FBN : jb_lo;
+  // key padding of this batch: keys outside [ks, ke) are never visible
+  const int ks = p.kv_start ? max(0, p.kv_start[n]) : 0;
+  const int ke = p.kv_end ? min(p.S, p.kv_end[n]) : p.S;
+  const int jb_lo = max(lo_blk, ks) / FBN;
+  const int jb_hi = min(hi_blk, ke) > max(lo_blk, ks) ? (min(hi_blk, ke) + FBN - 1) / FBN : jb_lo;
   // streaming: key blocks between the kept head and the first row's window are invisible to all rows
   const int gap_lo = (p.keep + FBN - 1) / FBN;
   const int gap_hi = (p.mask_kind == MASK_STREAM) ? max(0, r0 + off - p.window + 1) / FBN : 0;
@@ -165,6 +172,10 @@ __global__ void __launch_bounds__(FTHREADS) fp32_attn_kernel(const F32Params p) 
         const int key = k0 + cg + 8 * c;
         float zz = RBF ? (2.f * p.scale) * z[r][c] - p.scale * sm.kn[cg + 8 * c] : p.scale * z[r][c];
         if (key >= hi_i[r] || (key < lo_i[r] && key >= p.keep)) zz = -INFINITY;
+        if (key < ks || key >= ke) zz = -INFINITY;
+        if (p.mask_bits != nullptr && i < p.L && key < p.S &&
+            !((p.mask_bits[(size_t)i * p.mask_words + (key >> 5)] >> (key & 31)) & 1u))
+          zz = -INFINITY;
         if (p.bias != nullptr && i < p.L && key < p.S) zz += p.bias[(size_t)i * p.S + key];
         z[r][c] = zz;
         mt = fmaxf(mt, zz);
@@ -248,6 +259,10 @@ int launch_f32_impl(const AttnArgs& a, cudaStream_t stream) {
   p.window = a.window;
   p.keep = a.keep;
   p.scale = a.scale;
+  p.mask_bits = a.mask_bits;
+  p.kv_start = a.kv_start;
+  p.kv_end = a.kv_end;
+  p.mask_words = (a.S + 31) / 32;
   const int smem = sizeof(F32Smem<E, EV>);
   auto kern = fp32_attn_kernel<E, EV, RBF>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -13;

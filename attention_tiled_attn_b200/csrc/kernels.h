@@ -25,6 +25,9 @@ struct AttnArgs {
   int window;
   const float* bias;   // [L, S] or nullptr
   int keep;            // MASK_STREAM: number of initial keys always visible (0 otherwise)
+  const uint32_t* mask_bits;  // [L][ceil(S/32)] keep bits (bit j%32 of word j/32), or nullptr
+  const int* kv_start;        // [N] first non-padding key per batch, or nullptr (0)
+  const int* kv_end;          // [N] one past the last non-padding key per batch, or nullptr (S)
 };
 
 constexpr float LOG2E = 1.4426950408889634f;

@@ -119,18 +119,34 @@ struct TileInfo {
   int jb_lo, jb_hi;  // key-tile range [jb_lo, jb_hi)
 };
 
+// EXT variant only (a separate kernel argument, so PrefillParams stays as it is):
+// a boolean keep mask packed 32 keys per word, and per-batch key padding.
+struct PadArgs {
+  const uint32_t* bits;  // [L][words]: bit j % 32 of word j / 32 = key j may be attended; or nullptr
+  const int* kv_start;   // [N] first non-padding key, or nullptr (0)
+  const int* kv_end;     // [N] one past the last non-padding key, or nullptr (S)
+  int words;             // ceil(S / 32)
+};
+
 // Key-tile range of a query tile; with the streaming mask also the first tile
 // past the kept initial keys (*gap_lo) and the first tile of the window of the
 // tile's first row (*gap_hi): the tiles in between no row of the tile sees.
-__device__ __forceinline__ void tile_range(const PrefillParams& p, TileInfo& t, int* gap_lo, int* gap_hi) {
+// EXT: keys outside [ks, ke) are padding for this tile's batch.
+template <bool EXT>
+__device__ __forceinline__ void tile_range(const PrefillParams& p, TileInfo& t, int* gap_lo, int* gap_hi, int ks,
+                                           int ke) {
   t.jb_lo = t.jb_hi = 0;
   *gap_lo = *gap_hi = -1;
   if (!t.active) return;
   const int off = p.S - p.L;
   const int r_last = min(t.r0 + BM - 1, p.L - 1);
-  const int hi = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, r_last + off + 1);
+  int hi = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, r_last + off + 1);
   const int win_lo = max(0, t.r0 + off - p.window + 1);  // the first row's window start
-  const int lo = (p.mask_kind == MASK_WINDOW || (p.mask_kind == MASK_STREAM && p.keep == 0)) ? win_lo : 0;
+  int lo = (p.mask_kind == MASK_WINDOW || (p.mask_kind == MASK_STREAM && p.keep == 0)) ? win_lo : 0;
+  if constexpr (EXT) {
+    lo = max(lo, ks);
+    hi = min(hi, ke);
+  }
   if (hi <= lo) return;
   t.jb_lo = lo / BN;
   t.jb_hi = (hi + BN - 1) / BN;
@@ -163,6 +179,7 @@ struct Item {
   TileInfo tile[2];
   int u_lo, u_hi;
   int g_lo, g_hi;  // key tiles [g_lo, g_hi) of the union range are skipped (-1: none)
+  int ks, ke;      // EXT: the batch's non-padding keys [ks, ke)
 };
 
 // Next key tile of an item after jb.  With the streaming mask every role steps
@@ -174,7 +191,10 @@ __device__ __forceinline__ int next_jb(const Item& w, int jb) {
   return jb + 1;
 }
 
-__device__ __forceinline__ void decode_item(const PrefillParams& p, int item, Item& w) {
+// Both query tiles of an item belong to one batch, so key padding narrows their
+// ranges alike and the two key-tile lists still nest as the issuer needs.
+template <bool EXT>
+__device__ __forceinline__ void decode_item(const PrefillParams& p, const PadArgs& pa, int item, Item& w) {
   if (p.head_pairs) {
     const int hp_per = p.group / 2;
     const int per_rb = p.N * p.H * hp_per;
@@ -197,9 +217,15 @@ __device__ __forceinline__ void decode_item(const PrefillParams& p, int item, It
     w.tile[0] = {1, hq, 2 * rp * BM, 0, 0};
     w.tile[1] = {(2 * rp + 1) * BM < p.L ? 1 : 0, hq, (2 * rp + 1) * BM, 0, 0};
   }
+  w.ks = 0;
+  w.ke = p.S;
+  if constexpr (EXT) {
+    if (pa.kv_start) w.ks = max(0, __ldg(pa.kv_start + w.n));
+    if (pa.kv_end) w.ke = min(p.S, __ldg(pa.kv_end + w.n));
+  }
   int gl0, gh0, gl1, gh1;
-  tile_range(p, w.tile[0], &gl0, &gh0);
-  tile_range(p, w.tile[1], &gl1, &gh1);
+  tile_range<EXT>(p, w.tile[0], &gl0, &gh0, w.ks, w.ke);
+  tile_range<EXT>(p, w.tile[1], &gl1, &gh1, w.ks, w.ke);
   const bool h0 = w.tile[0].jb_hi > w.tile[0].jb_lo;
   const bool h1 = w.tile[1].jb_hi > w.tile[1].jb_lo;
   w.u_lo = w.u_hi = 0;
@@ -229,12 +255,13 @@ __device__ __forceinline__ void decode_item(const PrefillParams& p, int item, It
 // (k even) or k*G + G-1-b (k odd), so the heavy items spread evenly.
 __device__ __forceinline__ int snake_item(int b, int k, int G) { return k * G + ((k & 1) ? (G - 1 - b) : b); }
 
-// STREAM: the streaming mask with kept initial keys (a compile-time switch, so the
-// other masks carry none of its bookkeeping in the softmax warps' registers).
-template <int E, int EV, bool RBF, bool STREAM>
+// STREAM: the streaming mask with kept initial keys; EXT: keep bits and key padding
+// (compile-time switches, so the other masks carry none of their bookkeeping in
+// the softmax warps' registers).
+template <int E, int EV, bool RBF, bool STREAM, bool EXT>
 __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p, const PadArgs pa) {
   using C = Cfg<E, EV, RBF>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -298,7 +325,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
         const int item = snake_item(b, k, G);
         if (item >= p.n_items) continue;
         Item w;
-        decode_item(p, item, w);
+        decode_item<EXT>(p, pa, item, w);
         if (w.u_hi <= w.u_lo) continue;
         const bool h0 = w.tile[0].jb_hi > w.tile[0].jb_lo, h1 = w.tile[1].jb_hi > w.tile[1].jb_lo;
         bool q_pending = true;
@@ -357,7 +384,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
         const int item = snake_item(b, k, G);
         if (item >= p.n_items) continue;
         Item w;
-        decode_item(p, item, w);
+        decode_item<EXT>(p, pa, item, w);
         if (w.u_hi <= w.u_lo) continue;
         if (!wait_bar(bar(C::B_QFULL), qc & 1, abort_flag)) break;
         ++qc;
@@ -464,7 +491,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
       const int item = snake_item(b, k, G);
       if (item >= p.n_items) continue;
       Item w;
-      decode_item(p, item, w);
+      decode_item<EXT>(p, pa, item, w);
       for (int jb = w.u_lo; jb < w.u_hi; jb = next_jb<STREAM>(w, jb), ++gk) {
         const uint32_t ks = gk % C::NK;
         const uint32_t slot = gk % C::NKN;
@@ -511,7 +538,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t t_s = tmem + lane_base + t * 128;
     const uint32_t t_o = tmem + lane_base + 256 + t * EV;
-    const bool has_bias = p.bias != nullptr;
+    const bool has_bias = !EXT && p.bias != nullptr;  // the EXT entry takes keep bits instead
     const int off = p.S - p.L;
     uint32_t gk = 0;   // union key tiles seen (key-norm ring)
     uint32_t sc = 0;   // S tiles consumed (s_full / p_full phases)
@@ -521,14 +548,20 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
       const int item = snake_item(b, k, G);
       if (item >= p.n_items) continue;
       Item w;
-      decode_item(p, item, w);
+      decode_item<EXT>(p, pa, item, w);
       const TileInfo T = t ? w.tile[1] : w.tile[0];
       const int i = T.r0 + row;
       // key j visible to row i iff lo_i <= j < hi_i (streaming mask: or j < keep)
-      const int lo_i = (STREAM || p.mask_kind == MASK_WINDOW) ? (i + off - p.window + 1) : 0;
-      const int hi_i = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, i + off + 1);
-      const int first_row_hi = T.r0 + off + 1;  // key limit of the tile's first row
-      const int last_row_lo = min(T.r0 + BM - 1, p.L - 1) + off - p.window + 1;
+      int lo_i = (STREAM || p.mask_kind == MASK_WINDOW) ? (i + off - p.window + 1) : 0;
+      int hi_i = (p.mask_kind == MASK_NONE) ? p.S : min(p.S, i + off + 1);
+      int first_row_hi = T.r0 + off + 1;  // key limit of the tile's first row
+      int last_row_lo = min(T.r0 + BM - 1, p.L - 1) + off - p.window + 1;
+      if constexpr (EXT) {  // padding narrows every row's range; the bounds are the tile's extremes
+        lo_i = max(lo_i, w.ks);
+        hi_i = min(hi_i, w.ke);
+        first_row_hi = min(p.mask_kind == MASK_NONE ? p.S : first_row_hi, w.ke);
+        last_row_lo = max(p.mask_kind == MASK_WINDOW ? last_row_lo : 0, w.ks);
+      }
       const float* bias_row = has_bias && i < p.L ? p.bias + static_cast<size_t>(i) * p.S : nullptr;
 
       float m_run = -INFINITY, l_run = 0.f;
@@ -576,9 +609,12 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
         }
 
         const int k0 = jb * BN;
-        const bool need_mask = ((k0 + BN) > p.S) || (p.mask_kind != MASK_NONE && (k0 + BN) > first_row_hi) ||
-                               ((STREAM || p.mask_kind == MASK_WINDOW) && k0 < last_row_lo &&
-                                (!STREAM || k0 + BN > p.keep));
+        bool need_mask;
+        if constexpr (EXT)
+          need_mask = (k0 + BN) > first_row_hi || k0 < last_row_lo;
+        else
+          need_mask = ((k0 + BN) > p.S) || (p.mask_kind != MASK_NONE && (k0 + BN) > first_row_hi) ||
+                      ((STREAM || p.mask_kind == MASK_WINDOW) && k0 < last_row_lo && (!STREAM || k0 + BN > p.keep));
         // Logits stay in "exponent units" u with  base-2 logit = u * c_exp:
         //   dot: u = q.k (+ bias / scale),  c_exp = scale * log2e
         //   rbf: u = 2*scale*log2e*q.k - scale*log2e*||k||^2 (+ bias * log2e),  c_exp = 1
@@ -610,6 +646,22 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
 #pragma unroll
             for (int c = 0; c < BN; ++c)
               if (c < lo || c >= hi) z[c] = -INFINITY;
+          }
+        }
+        if constexpr (EXT) {
+          // keep bits of this row's 128 keys (words past the row's end read as 0: keys >= S are masked anyway)
+          if (pa.bits != nullptr && i < p.L) {
+            const uint32_t* brow = pa.bits + static_cast<size_t>(i) * pa.words + (k0 >> 5);
+            const int wl = pa.words - (k0 >> 5);
+            const uint32_t m0 = __ldg(brow), m1 = wl > 1 ? __ldg(brow + 1) : 0u;
+            const uint32_t m2 = wl > 2 ? __ldg(brow + 2) : 0u, m3 = wl > 3 ? __ldg(brow + 3) : 0u;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (!((m0 >> c) & 1u)) z[c] = -INFINITY;
+              if (!((m1 >> c) & 1u)) z[32 + c] = -INFINITY;
+              if (!((m2 >> c) & 1u)) z[64 + c] = -INFINITY;
+              if (!((m3 >> c) & 1u)) z[96 + c] = -INFINITY;
+            }
           }
         }
         if (has_bias && bias_row != nullptr) {
@@ -748,7 +800,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-template <int E, int EV, bool RBF, bool STREAM>
+template <int E, int EV, bool RBF, bool STREAM, bool EXT>
 int launch_impl(const AttnArgs& a, cudaStream_t stream) {
   using C = Cfg<E, EV, RBF>;
   CUtensorMap tq, tk, tv;
@@ -781,7 +833,12 @@ int launch_impl(const AttnArgs& a, cudaStream_t stream) {
   p.c_kn = a.scale * LOG2E;
   p.c_exp = RBF ? 1.f : a.scale * LOG2E;
   p.c_bias = RBF ? LOG2E : 1.f / a.scale;
-  auto kern = prefill_kernel<E, EV, RBF, STREAM>;
+  PadArgs pa{};
+  pa.bits = a.mask_bits;
+  pa.kv_start = a.kv_start;
+  pa.kv_end = a.kv_end;
+  pa.words = (a.S + 31) / 32;
+  auto kern = prefill_kernel<E, EV, RBF, STREAM, EXT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return -13;
   {
@@ -793,7 +850,7 @@ int launch_impl(const AttnArgs& a, cudaStream_t stream) {
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return -13;
   const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: one CTA per SM
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p, pa);
   return cudaGetLastError() == cudaSuccess ? 0 : -13;
 }
 
@@ -820,10 +877,12 @@ unsigned int take_status_prefill(cudaStream_t s) { return take_device_status_loc
 int launch_prefill_bf16(const AttnArgs& a, cudaStream_t stream) {
   const bool r = a.rbf;
   const bool st = a.mask_kind == MASK_STREAM && a.keep > 0;
-#define ATTN_PREFILL_CASE(e, ev)                                                                 \
-  if (a.E == e && a.Ev == ev) {                                                                  \
-    if (st) return r ? launch_impl<e, ev, true, true>(a, stream) : launch_impl<e, ev, false, true>(a, stream); \
-    return r ? launch_impl<e, ev, true, false>(a, stream) : launch_impl<e, ev, false, false>(a, stream); \
+  const bool ext = a.mask_bits != nullptr || a.kv_start != nullptr || a.kv_end != nullptr;
+#define ATTN_PREFILL_CASE(e, ev)                                                                              \
+  if (a.E == e && a.Ev == ev) {                                                                               \
+    if (st) return r ? launch_impl<e, ev, true, true, false>(a, stream) : launch_impl<e, ev, false, true, false>(a, stream); \
+    if (ext) return r ? launch_impl<e, ev, true, false, true>(a, stream) : launch_impl<e, ev, false, false, true>(a, stream); \
+    return r ? launch_impl<e, ev, true, false, false>(a, stream) : launch_impl<e, ev, false, false, false>(a, stream); \
   }
   ATTN_PREFILL_CASE(64, 64)
   ATTN_PREFILL_CASE(128, 128)

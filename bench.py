@@ -78,8 +78,28 @@ def row_pairs(r: sw.Recipe, rows) -> np.ndarray:
 
 
 def visible_pairs(r: sw.Recipe) -> int:
-    """Number of (query, key) pairs the mask leaves visible, per (n, hq)."""
+    """Number of (query, key) pairs the mask leaves visible, per (n, hq) (no keep bits or padding)."""
     return int(row_pairs(r, np.arange(r.L)).sum())
+
+
+def visible_pairs_total(r: sw.Recipe) -> int:
+    """Visible (query, key) pairs summed over the batch, per query head: the mask kind,
+    then the keep bits and each batch's key padding."""
+    ks, ke = sw.kv_ranges(r)
+    keep = sw.keep_matrix(r)
+    if keep is None and ks is None:
+        return r.N * visible_pairs(r)
+    ip = np.arange(r.L, dtype=np.int64) + (r.S - r.L)
+    hi = np.full(r.L, r.S) if r.mask_kind == "none" else np.minimum(r.S, ip + 1)
+    lo = np.maximum(0, ip - r.window + 1) if r.mask_kind == "window" else np.zeros(r.L, dtype=np.int64)
+    starts = np.zeros(r.N, dtype=np.int64) if ks is None else ks.astype(np.int64)
+    ends = np.full(r.N, r.S) if ke is None else ke.astype(np.int64)
+    if keep is None:
+        return int(sum(np.maximum(0, np.minimum(hi, e) - np.maximum(lo, b)).sum() for b, e in zip(starts, ends)))
+    j = np.arange(r.S)[None, :]
+    vis = keep & (j >= lo[:, None]) & (j < hi[:, None])
+    csum = np.concatenate([np.zeros((r.L, 1), dtype=np.int64), np.cumsum(vis, axis=1)], axis=1)
+    return int(sum((csum[:, e] - csum[:, b]).sum() for b, e in zip(starts, ends)))
 
 
 def is_decode(r: sw.Recipe) -> bool:
@@ -107,7 +127,7 @@ def work_units(r: sw.Recipe):
     if is_decode(r):
         kv_bytes = r.N * r.H * decode_keys(r) * (r.E + r.Ev) * 2
         return kv_bytes, "GB/s", "hbm"
-    flops = 2 * (r.E + r.Ev) * visible_pairs(r) * r.N * r.Hq
+    flops = 2 * (r.E + r.Ev) * visible_pairs_total(r) * r.Hq
     return flops, "TFLOP/s", "tensor"
 
 
@@ -259,7 +279,8 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
                                      stream=stream)
             return
         attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=r.mode, sink=t["sink"], mask_kind=r.mask_kind,
-                      window=r.window, keep_first=r.keep, bias=t["bias"], out=out, lse=lse, stream=stream)
+                      window=r.window, keep_first=r.keep, bias=t["bias"], out=out, lse=lse, stream=stream,
+                      mask_bits=t["mask_bits"], kv_start=t["kv_start"], kv_end=t["kv_end"])
 
     amount, unit, bound = work_units(r)
     barrier(pg)
@@ -325,7 +346,8 @@ def e2e_measure(res, steps, warmup):
         else:
             attn.attn_fwd(dev["q"], dev["k"], dev["v"], scale=r.scale, mode=r.mode, sink=t["sink"],
                           mask_kind=r.mask_kind, window=r.window, keep_first=r.keep, bias=t["bias"], out=res["out"],
-                          lse=res["lse"], stream=stream)
+                          lse=res["lse"], stream=stream, mask_bits=t["mask_bits"], kv_start=t["kv_start"],
+                          kv_end=t["kv_end"])
         out_host.copy_(res["out"], non_blocking=True)
         lse_host.copy_(res["lse"], non_blocking=True)
 
@@ -449,6 +471,10 @@ def ours(args):
         if base.mode == "dot" and base.dtype == "bf16" and not is_decode(base):
             runs.append((args.workload + ":steady_state_noncausal_8k",
                          dataclasses.replace(base, N=1, L=8192, S=8192, mask_kind="none")))
+            # a 10% random 0/-inf mask as packed keep bits and as the fp32 bias; ragged left padding
+            runs.append((args.workload + ":keep_bits_random10", dataclasses.replace(base, keep_mask="random10")))
+            runs.append((args.workload + ":bias_random10", dataclasses.replace(base, bias="random10")))
+            runs.append((args.workload + ":left_pad_upto50", dataclasses.replace(base, pad_left=0.5)))
         for name in names:
             r0 = sw.RECIPES[name]
             runs.append((name, r0))
@@ -489,6 +515,10 @@ def ours(args):
                 if ctl in extra:
                     extra[label]["time_vs_" + ctl.split(":")[1]] = round(
                         extra[label]["ms_per_step"] / extra[ctl]["ms_per_step"], 4)
+            if label + ":keep_bits_random10" in extra and label + ":bias_random10" in extra:
+                extra[label + ":keep_bits_random10"]["time_vs_bias"] = round(
+                    extra[label + ":keep_bits_random10"]["ms_per_step"] / extra[label + ":bias_random10"]["ms_per_step"],
+                    4)
             if label + ":top_k_33x" in extra:
                 extra[label + ":top_k_33x"]["time_vs_dense"] = round(
                     extra[label + ":top_k_33x"]["ms_per_step"] / extra[label]["ms_per_step"], 4)

@@ -127,6 +127,37 @@ int attn_fwd_streaming(const void* q, const void* k, const void* v, void* out, f
                        int dtype, void* stream);
 
 /*
+ * attn_fwd_padded -- attn_fwd with a packed boolean keep mask and per-batch key
+ * padding in place of the float bias (page "SDPA란 무엇인가" §1: B holds 0 or
+ * -inf; §4 trap 1: in a boolean attn_mask, True marks a pair that takes part;
+ * the page's left-padding check: with the mask passed, padded and unpadded
+ * inputs give the same output on the real tokens).
+ *
+ *   mask_bits  [L, ceil(S/32)] uint32, device, or NULL (every pair kept): bit
+ *              j % 32 of word i*ceil(S/32) + j/32 set means query row i may
+ *              attend to key j.  Broadcast over batch and heads.  32x fewer
+ *              bytes than the equivalent float bias.
+ *   kv_start   [N] int32, device, or NULL (0): keys j < kv_start[n] are padding
+ *              for batch n (left padding).
+ *   kv_end     [N] int32, device, or NULL (S): keys j >= kv_end[n] are padding
+ *              (right padding / variable length).  Values are clamped to
+ *              [0, S]; kv_start >= kv_end leaves batch n no key.
+ *
+ * Key j is visible to row i of batch n iff the mask kind allows it, its bit is
+ * set, and kv_start[n] <= j < kv_end[n].  A row with no visible key gets out = 0
+ * and lse = -inf (lse = s with a sink), as SDPA does for left-padded start rows.
+ * Tiles of keys wholly inside the padding are not read.  All other arguments,
+ * layouts, ownership, dispatch and status codes are attn_fwd's (mask_kind is
+ * NONE, CAUSAL or SLIDING_WINDOW); mask_bits, kv_start and kv_end must be
+ * 4-byte aligned (ATTN_ERR_ALIGNMENT).
+ */
+int attn_fwd_padded(const void* q, const void* k, const void* v, void* out, float* lse,
+                    int N, int Hq, int H, int L, int S, int E, int Ev, float scale, int mode,
+                    const float* sink_logits, int mask_kind, int window,
+                    const unsigned int* mask_bits, const int* kv_start, const int* kv_end,
+                    int dtype, void* stream);
+
+/*
  * attn_decode_indexed -- exact decode attention over a listed subset of the
  * cached keys: the step that follows a top-k key selection (page "기술 요약:
  * SOCKET - 희소 어텐션을 위한 SOft Collision Kernel EsTimator", 방법론, 핵심

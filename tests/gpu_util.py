@@ -31,7 +31,8 @@ def run_gpu(r: sw.Recipe, t: dict):
         torch.cuda.synchronize()
         return out, lse
     out, lse = attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=api_mode(r), sink=t["sink"],
-                             mask_kind=r.mask_kind, window=r.window, bias=t["bias"], keep_first=r.keep)
+                             mask_kind=r.mask_kind, window=r.window, bias=t["bias"], keep_first=r.keep,
+                             mask_bits=t.get("mask_bits"), kv_start=t.get("kv_start"), kv_end=t.get("kv_end"))
     torch.cuda.synchronize()
     return out, lse
 
@@ -69,8 +70,12 @@ def oracle_rows(r: sw.Recipe, n: int, hq: int, rows, host: dict | None = None):
     bias = sw.bias_matrix(r)
     s = None if sink is None else float(sink[hq])
     b = None if bias is None else bias[rows].astype(np.float64)
+    km = sw.keep_matrix(r)
+    ks, ke = sw.kv_ranges(r)
+    rng = None if ks is None else (int(ks[n]), int(ke[n]))
     return orc.attend_rows(q[rows], rows, k, v, r.L, scale=r.scale, mode=r.mode, sink=s,
-                           mask_kind=r.mask_kind, window=r.window, bias_rows=b, keep=r.keep)
+                           mask_kind=r.mask_kind, window=r.window, bias_rows=b, keep=r.keep,
+                           keep_rows=None if km is None else km[rows], kv_range=rng)
 
 
 def compare(r: sw.Recipe, got_out, got_lse, ref_out, ref_lse, what=""):
@@ -119,11 +124,17 @@ def run_and_check_full(r: sw.Recipe, key_idx: np.ndarray | None = None):
             sink=None if host["sink"] is None else host["sink"].astype(np.float64), mask_kind=r.mask_kind,
             window=r.window, bias=None if host["bias"] is None else host["bias"].astype(np.float64))
         return compare(r, out_to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, r.name)
+    if host["keep"] is not None:
+        t["mask_bits"] = torch.from_numpy(sw.pack_mask_bits(host["keep"]).view(np.int32)).cuda()
+    if host["kv_start"] is not None:
+        t["kv_start"] = torch.from_numpy(host["kv_start"]).cuda()
+        t["kv_end"] = torch.from_numpy(host["kv_end"]).cuda()
     out, lse = run_gpu(r, t)
     ref_out, ref_lse = orc.attention_forward(
         sw.as_f64(r, host["q"]), sw.as_f64(r, host["k"]), sw.as_f64(r, host["v"]), scale=r.scale, mode=r.mode,
         sink=None if host["sink"] is None else host["sink"].astype(np.float64), mask_kind=r.mask_kind,
-        window=r.window, bias=None if host["bias"] is None else host["bias"].astype(np.float64), keep=r.keep)
+        window=r.window, bias=None if host["bias"] is None else host["bias"].astype(np.float64), keep=r.keep,
+        mask_keep=host["keep"], kv_start=host["kv_start"], kv_end=host["kv_end"])
     return compare(r, out_to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, r.name)
 
 

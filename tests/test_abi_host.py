@@ -114,6 +114,25 @@ def test_indexed_argument_validation(lib, kw, status):
     assert call_indexed(**kw) == status
 
 
+def call_padded(**kw):
+    a = dict(q=P, k=P, v=P, out=P, lse=P, N=1, Hq=2, H=1, L=8, S=8, E=64, Ev=64, scale=0.125, mode=0,
+             sink=None, mask_kind=1, window=0, bits=P, start=P, end=P, dtype=0, stream=None)
+    a.update(kw)
+    return attn.attn_fwd_padded_raw(a["q"], a["k"], a["v"], a["out"], a["lse"], a["N"], a["Hq"], a["H"], a["L"],
+                                    a["S"], a["E"], a["Ev"], a["scale"], a["mode"], a["sink"], a["mask_kind"],
+                                    a["window"], a["bits"], a["start"], a["end"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(mask_kind=3), -7), (dict(mask_kind=2, window=0), -8),
+    (dict(bits=P + 2), -11), (dict(start=P + 1), -11), (dict(end=P + 3), -11),
+    (dict(q=None), -1), (dict(Hq=3, H=2), -3), (dict(E=96), -4), (dict(scale=-1.0), -5), (dict(mode=2), -9),
+    (dict(dtype=5), -10),
+])
+def test_padded_argument_validation(lib, kw, status):
+    assert call_padded(**kw) == status
+
+
 def test_python_binding_rejects_cpu_tensors(lib):
     import torch
     q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)

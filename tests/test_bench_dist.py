@@ -86,3 +86,26 @@ def test_visible_pairs_and_decode_keys_match_the_oracle_mask():
             assert bench.visible_pairs(r) == int(vis.sum()), (L, S, mk, w, keep)
             if mk in ("window", "streaming"):
                 assert bench.decode_keys(r) == int(vis.any(axis=0).sum()), (L, S, mk, w, keep)
+
+
+def test_visible_pairs_total_with_keep_bits_and_padding():
+    """Work accounting with keep bits and ragged padding equals the oracle's visibility count."""
+    import dataclasses
+
+    import numpy as np
+
+    from oracle import attention as orc
+    from synth import workloads as sw
+    base = sw.RECIPES["tiny_rbf_sink_causal_f32"]
+    for mk, w in (("none", 0), ("causal", 0), ("window", 9)):
+        for keep, pl, pr in (("random10", 0.0, 0.0), ("none", 0.5, 0.0), ("random10", 0.3, 0.4), ("none", 0.0, 0.6)):
+            r = dataclasses.replace(base, N=5, L=40, S=61, mask_kind=mk, window=w, keep_mask=keep, pad_left=pl,
+                                    pad_right=pr)
+            km = sw.keep_matrix(r)
+            ks, ke = sw.kv_ranges(r)
+            want = 0
+            for n in range(r.N):
+                vis = orc.padded_visible(orc.visible(np.arange(r.L), r.S, r.L, mk, w), km,
+                                         None if ks is None else (ks[n], ke[n]))
+                want += int(vis.sum())
+            assert bench.visible_pairs_total(r) == want, (mk, keep, pl, pr)

@@ -97,6 +97,50 @@ DECODE_CASES = [
 ]
 
 
+# packed keep bits and per-batch key padding (attn_fwd_padded), on every path
+PADDED_CASES = [
+    R("pd_keep_causal_300_g2_e128", L=300, S=300, E=128, Ev=128, Hq=4, H=2, mask_kind="causal",
+      keep_mask="random10", sink="normal"),
+    R("pd_left_pad_causal_600", L=600, S=600, N=3, mask_kind="causal", pad_left=0.5),
+    R("pd_right_pad_none_500_e128", L=500, S=500, N=2, E=128, Ev=128, pad_right=0.4, sink="normal"),
+    R("pd_rbf_window_keep_both_pads_700", L=700, S=700, N=2, mode="rbf", mask_kind="window", window=100,
+      keep_mask="random10", pad_left=0.3, pad_right=0.3),
+    R("pd_keep_none_L200_S1000", L=200, S=1000, keep_mask="random10", pad_left=0.2),
+    R("pd_keep_S130_ragged_words", L=130, S=130, Hq=6, H=2, keep_mask="random10", mask_kind="causal"),
+    R("f_pd_keep_left_causal_f32", L=150, S=170, Hq=3, H=1, dtype="f32", mask_kind="causal", keep_mask="random10",
+      pad_left=0.4, sink="normal"),
+    R("f_pd_right_window_rbf_f32", L=100, S=300, N=2, dtype="f32", mode="rbf", mask_kind="window", window=60,
+      pad_right=0.5),
+    R("d_pd_keep_L2_S777", L=2, S=777, Hq=4, H=2, keep_mask="random10", sink="normal"),
+    R("d_pd_left_L1_S5000", L=1, S=5000, N=4, Hq=8, H=2, E=128, Ev=128, pad_left=0.5, scale=0.0884),
+    R("d_pd_right_L4_g4_causal", L=4, S=900, N=3, Hq=8, H=2, mask_kind="causal", pad_right=0.6, keep_mask="random10"),
+]
+
+
+@pytest.mark.parametrize("r", PADDED_CASES, ids=lambda r: r.name)
+def test_padded_small(r):
+    gu.run_and_check_full(r)
+
+
+def test_padded_start_beyond_end_masks_everything():
+    """kv_start >= kv_end leaves the batch no key: out 0, lse -inf (or the sink)."""
+    for sink in ("none", "normal"):
+        r = R("pd_empty", L=130, S=130, N=2, Hq=2, H=2, sink=sink, pad_left=0.9)
+        host = sw.generate(r)
+        t = {x: sgpu.to_device(host[x], r) for x in ("q", "k", "v")}
+        t["sink"] = None if host["sink"] is None else torch.from_numpy(host["sink"]).cuda()
+        t["bias"] = None
+        t["kv_start"] = torch.tensor([120, 7], dtype=torch.int32, device="cuda")
+        t["kv_end"] = torch.tensor([60, 7], dtype=torch.int32, device="cuda")
+        out, lse = gu.run_gpu(r, t)
+        assert torch.all(out == 0)
+        want = float("-inf") if host["sink"] is None else None
+        for hq in range(r.Hq):
+            col = lse[:, hq].cpu().numpy()
+            exp = want if want is not None else float(host["sink"][hq])
+            assert np.all(col == exp) if want is not None else np.allclose(col, exp, atol=1e-6)
+
+
 # exact decode over a listed key subset (a top-k selection's output)
 INDEXED_CASES = [
     R("ix_L1_g4_S1000_sel100_sink", L=1, S=1000, E=128, Ev=128, N=2, Hq=8, H=2, n_sel=100, sink="normal",

@@ -40,6 +40,11 @@ in blocks of query rows so that memory stays bounded:
   mask passed, padded and unpadded inputs give the same output for the real
   tokens): key j is visible to row i only where keep[i, j] is True and, for
   batch n, kv_start[n] <= j < kv_end[n].  Both compose with every mask kind.
+* Backward (page "Attention Sink" §4.2 and §5: the sinks and register tokens
+  are learned parameters, so training needs gradients of q, k, v and the sink
+  logit; page "Dot-Product Attention을 거리 기반 RBF-Attention으로 교체한
+  실험기": the RBF model is trained): the chain rule through the definitions
+  above, written out in ``attention_backward``.
 * Exact attention over a selected key subset (page "기술 요약: SOCKET - 희소
   어텐션을 위한 SOft Collision Kernel EsTimator", 방법론, 핵심 메커니즘 step 4:
   the top-k keys are picked, then exact attention runs on that subset): the
@@ -231,3 +236,74 @@ def attention_over_index_set(q, k, v, key_idx, *, scale, sink=None, mask_kind="n
             out[n, hq] = alpha @ v[n, kvh][pos]
             lse[n, hq] = l
     return out, lse
+
+
+def softmax_grad(P: np.ndarray, dP: np.ndarray, D: np.ndarray) -> np.ndarray:
+    """dS_ij = P_ij (dP_ij - D_i): the gradient through the row softmax."""
+    return P * (dP - D[:, None])
+
+
+def score_input_grads(dS: np.ndarray, q_rows: np.ndarray, k: np.ndarray, scale: float, mode: str):
+    """(dq, dk) of one head from the logit gradients dS (R, S)."""
+    if mode == "dot":
+        return scale * dS @ k, scale * dS.T @ q_rows
+    return 2.0 * scale * dS @ k, 2.0 * scale * (dS.T @ q_rows - k * dS.sum(axis=0)[:, None])
+
+
+def sink_grad(p_sink: np.ndarray, D: np.ndarray) -> float:
+    """d loss / d s for one head: -sum_i p_i D_i."""
+    return -float(np.sum(p_sink * D))
+
+
+def attention_backward(q, k, v, dout, *, scale, mode="dot", sink=None, mask_kind="none", window=0, bias=None,
+                       keep=0):
+    """Gradients of the forward with respect to q, k, v and the sink logits.
+
+    The chain rule through the definitions above, in float64 and in this order
+    (row i, key j of one (batch, query head); P and D from the forward):
+      P_ij  = exp(z_ij - lse_i) on visible keys, 0 elsewhere
+      D_i   = sum_e dout_ie * out_ie
+      dV_j += sum_i P_ij dout_i                       (summed over the KV group)
+      dP_ij = dout_i . v_j
+      dS_ij = P_ij (dP_ij - D_i)
+      dot:  dQ_i = scale sum_j dS_ij k_j,   dK_j += scale sum_i dS_ij q_i
+      rbf:  z_ij = 2 scale q_i.k_j - scale |k_j|^2 (the logit frame above), so
+            dQ_i = 2 scale sum_j dS_ij k_j,  dK_j += 2 scale (sum_i dS_ij q_i - k_j sum_i dS_ij)
+      sink: the sink's share p_i = exp(s - lse_i) gives d out_i / d s = -p_i out_i,
+            so dsink_h = -sum_i p_i D_i (summed over batch and rows).
+    q, k, v, dout float64 arrays as in attention_forward.  Returns dq, dk, dv
+    (shapes of q, k, v) and dsink (Hq,) (zeros without a sink).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    N, Hq, L, _ = q.shape
+    H, S = k.shape[1], k.shape[2]
+    g = Hq // H
+    out, lse = attention_forward(q, k, v, scale=scale, mode=mode, sink=sink, mask_kind=mask_kind, window=window,
+                                 bias=bias, keep=keep)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dsink = np.zeros(Hq, dtype=np.float64)
+    rows = np.arange(L)
+    vis = visible(rows, S, L, mask_kind, window, keep)
+    for n in range(N):
+        for hq in range(Hq):
+            kvh = hq // g
+            z = logits(q[n, hq], k[n, kvh], scale, mode)
+            if bias is not None:
+                z = z + np.asarray(bias, dtype=np.float64)
+            l = lse[n, hq][:, None]
+            live = np.isfinite(l)
+            P = np.where(vis & np.isfinite(z) & live, np.exp(np.where(live, z - l, 0.0)), 0.0)
+            D = np.einsum("ie,ie->i", dout[n, hq], out[n, hq])
+            dv[n, kvh] += P.T @ dout[n, hq]
+            dP = dout[n, hq] @ v[n, kvh].T
+            dS = softmax_grad(P, dP, D)
+            gq, gk = score_input_grads(dS, q[n, hq], k[n, kvh], scale, mode)
+            dq[n, hq] = gq
+            dk[n, kvh] += gk
+            if sink is not None:
+                ps = np.where(live[:, 0], np.exp(float(sink[hq]) - np.where(live[:, 0], lse[n, hq], 0.0)), 0.0)
+                dsink[hq] += sink_grad(ps, D)
+    return dq, dk, dv, dsink

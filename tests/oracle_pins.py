@@ -484,10 +484,75 @@ def check_padding_and_keep_mask(seed=16):
     assert np.allclose(end[0], cut[0], atol=1e-13) and np.allclose(end[1], cut[1], atol=1e-13)
 
 
+def check_backward_finite_differences(seed=17):
+    """Every gradient of attention_backward against central differences of the
+    forward (loss = sum(out * W)), for both score modes, three mask kinds, with
+    and without a sink, under GQA: the differences involve none of the backward's
+    formulas."""
+    rng = np.random.default_rng(seed)
+    N, Hq, H, L, S, E, Ev = 2, 2, 1, 4, 6, 3, 2
+    h = 1e-6
+    for mode in ("dot", "rbf"):
+        for mk, W in (("none", 0), ("causal", 0), ("window", 3)):
+            for with_sink in (False, True):
+                q, k, v = _rand(rng, N, Hq, L, E), _rand(rng, N, H, S, E), _rand(rng, N, H, S, Ev)
+                Wt = _rand(rng, N, Hq, L, Ev)
+                sink = rng.standard_normal(Hq) if with_sink else None
+                kw = dict(scale=0.7, mode=mode, mask_kind=mk, window=W)
+
+                def loss(q_, k_, v_, s_):
+                    o, _ = orc.attention_forward(q_, k_, v_, sink=s_, **kw)
+                    return float(np.sum(o * Wt))
+
+                dq, dk, dv, ds = orc.attention_backward(q, k, v, Wt, sink=sink, **kw)
+                for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+                    it = np.nditer(arr, flags=["multi_index"])
+                    for _ in it:
+                        idx = it.multi_index
+                        a, b = arr.copy(), arr.copy()
+                        a[idx] += h
+                        b[idx] -= h
+                        args_a = {"q": (a, k, v), "k": (q, a, v), "v": (q, k, a)}[name]
+                        args_b = {"q": (b, k, v), "k": (q, b, v), "v": (q, k, b)}[name]
+                        fd = (loss(*args_a, sink) - loss(*args_b, sink)) / (2 * h)
+                        assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (mode, mk, with_sink, name, idx,
+                                                                                 fd, grad[idx])
+                if with_sink:
+                    for hh in range(Hq):
+                        sa, sb = sink.copy(), sink.copy()
+                        sa[hh] += h
+                        sb[hh] -= h
+                        fd = (loss(q, k, v, sa) - loss(q, k, v, sb)) / (2 * h)
+                        assert abs(fd - ds[hh]) <= 1e-6 * max(1.0, abs(fd)), (mode, mk, "sink", hh)
+                else:
+                    assert np.all(ds == 0.0)
+
+
+def check_backward_matches_sdpa_autograd(seed=18):
+    """Dot mode without a sink: the gradients equal PyTorch's SDPA autograd in
+    float64 (no mask, bottom-right causal, and an additive 0/-inf bias)."""
+    rng = np.random.default_rng(seed)
+    N, H, L, S, E, Ev = 2, 3, 5, 9, 4, 6
+    q, k, v = _rand(rng, N, H, L, E), _rand(rng, N, H, S, E), _rand(rng, N, H, S, Ev)
+    dout = _rand(rng, N, H, L, Ev)
+    bias = np.where(rng.random((L, S)) < 0.2, -np.inf, 0.0)
+    bias[:, -1] = 0.0
+    for mk, mask in (("none", None), ("causal", causal_lower_right(L, S)), ("bias", bias)):
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+        am = torch.tensor(mask) if mk == "bias" else mask
+        out = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=am, scale=0.5)
+        out.backward(torch.tensor(dout))
+        dq, dk, dv, _ = orc.attention_backward(q, k, v, dout, scale=0.5, mask_kind="causal" if mk == "causal" else "none",
+                                               bias=bias if mk == "bias" else None)
+        for got, want in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+            assert np.allclose(got, want.numpy(), atol=1e-12), mk
+
+
 ALL_CHECKS = [
     check_dot_matches_sdpa, check_brute_force, check_rbf_expansion, check_rbf_limits,
     check_dot_limits, check_uniform_entropy_golden, check_sink_limit, check_sink_mass,
     check_zero_sink_equivalence, check_convexity, check_causal_alignment_golden,
     check_fully_masked_rows, check_window_semantics, check_permutation_equivariance,
     check_gqa_repeat, check_streaming_mask, check_index_set, check_padding_and_keep_mask,
+    check_backward_finite_differences, check_backward_matches_sdpa_autograd,
 ]

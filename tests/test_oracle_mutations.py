@@ -101,7 +101,35 @@ def _padding_end_inclusive(vis, keep_rows=None, kv_range=None):
     return _real_padded_visible(vis, keep_rows, wide)
 
 
+_real_score_grads = orc.score_input_grads
+
+
+def _softmax_grad_no_D(P, dP, D):
+    return P * dP  # drops the -D_i term
+
+
+def _rbf_grad_without_norm_term(dS, q_rows, k, scale, mode):
+    if mode == "rbf":
+        return 2.0 * scale * dS @ k, 2.0 * scale * dS.T @ q_rows  # drops -k_j sum_i dS_ij
+    return _real_score_grads(dS, q_rows, k, scale, mode)
+
+
+def _dot_grad_unscaled(dS, q_rows, k, scale, mode):
+    if mode == "dot":
+        return dS @ k, dS.T @ q_rows
+    return _real_score_grads(dS, q_rows, k, scale, mode)
+
+
+def _sink_grad_sign(p_sink, D):
+    return float(np.sum(p_sink * D))
+
+
 MUTATIONS = [
+    ("softmax_grad", _softmax_grad_no_D, pins.check_backward_finite_differences),
+    ("softmax_grad", _softmax_grad_no_D, pins.check_backward_matches_sdpa_autograd),
+    ("score_input_grads", _rbf_grad_without_norm_term, pins.check_backward_finite_differences),
+    ("score_input_grads", _dot_grad_unscaled, pins.check_backward_matches_sdpa_autograd),
+    ("sink_grad", _sink_grad_sign, pins.check_backward_finite_differences),
     ("padded_visible", _padding_range_ignored, pins.check_padding_and_keep_mask),
     ("padded_visible", _keep_mask_inverted, pins.check_padding_and_keep_mask),
     ("padded_visible", _padding_end_inclusive, pins.check_padding_and_keep_mask),

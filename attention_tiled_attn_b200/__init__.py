@@ -54,6 +54,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_fwd_padded.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp, vp, vp, ci,
                                     vp]
     lib.attn_fwd_padded.restype = ci
+    lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp]
+    lib.attn_bwd.restype = ci
     lib.attn_status_string.argtypes = [ci]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_release_workspace.argtypes = []
@@ -93,6 +95,51 @@ def attn_fwd_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H, L, S, E, Ev, s
     return lib.attn_fwd(c(q_ptr), c(k_ptr), c(v_ptr), c(out_ptr), c(lse_ptr), int(N), int(Hq), int(H), int(L),
                         int(S), int(E), int(Ev), float(scale), int(mode), c(sink_ptr), int(mask_kind),
                         int(window), c(bias_ptr), int(dtype), c(stream_ptr))
+
+
+def attn_bwd_raw(q_ptr, k_ptr, v_ptr, out_ptr, dout_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr, dsink_ptr, N, Hq, H, L, S,
+                 E, Ev, scale, mode, sink_ptr, mask_kind, window, stream_ptr) -> int:
+    """The backward C entry point with integer pointers; returns the status code."""
+    lib = load_library()
+    c = lambda p: None if p is None else ctypes.c_void_p(int(p))  # noqa: E731
+    return lib.attn_bwd(c(q_ptr), c(k_ptr), c(v_ptr), c(out_ptr), c(dout_ptr), c(lse_ptr), c(dq_ptr), c(dk_ptr),
+                        c(dv_ptr), c(dsink_ptr), int(N), int(Hq), int(H), int(L), int(S), int(E), int(Ev),
+                        float(scale), int(mode), c(sink_ptr), int(mask_kind), int(window), c(stream_ptr))
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+             dout: torch.Tensor, *, scale: float, mode: str = "dot", sink: torch.Tensor | None = None,
+             mask_kind: str = "none", window: int = 0, stream: torch.cuda.Stream | None = None):
+    """Gradients (dq, dk, dv, dsink) of attn_fwd's output; float32 tensors, dsink None without a sink.
+
+    q, k, v, out, dout: contiguous bfloat16 CUDA tensors (the forward's inputs and
+    output, and the loss gradient of the output); lse: the forward's float32 lse.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D bfloat16 CUDA tensor")
+    N, Hq, L, E = q.shape
+    _, H, S, _ = k.shape
+    Ev = v.shape[3]
+    if tuple(out.shape) != (N, Hq, L, Ev) or tuple(dout.shape) != (N, Hq, L, Ev):
+        raise ValueError("out and dout must be (N, Hq, L, Ev)")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (N, Hq, L) or not lse.is_cuda or not lse.is_contiguous():
+        raise ValueError("lse must be the forward's float32 (N, Hq, L) tensor")
+    if sink is not None and (sink.dtype != torch.float32 or sink.numel() != Hq or not sink.is_cuda
+                             or not sink.is_contiguous()):
+        raise ValueError("sink must be a contiguous CUDA float32 tensor of Hq values")
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    dsink = torch.empty(Hq, dtype=torch.float32, device=q.device) if sink is not None else None
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = load_library().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                     _ptr(dv), _ptr(dsink), N, Hq, H, L, S, E, Ev, float(scale), MODES[mode],
+                                     _ptr(sink), MASKS[mask_kind], int(window), ctypes.c_void_p(stream.cuda_stream))
+    _check(st)
+    return dq, dk, dv, dsink
 
 
 def attn_fwd_padded_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H, L, S, E, Ev, scale, mode, sink_ptr,

@@ -22,7 +22,7 @@ BUILD_DIR = os.path.join(HERE, "_build")
 LIB_DIR = os.path.join(HERE, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libattn_b200.so")
 
-SOURCES = ["attn_abi.cu", "prefill_sm100.cu", "decode_sm100.cu", "fp32_simt.cu", "decode_noalloc.cu"]
+SOURCES = ["attn_abi.cu", "prefill_sm100.cu", "decode_sm100.cu", "fp32_simt.cu", "decode_noalloc.cu", "bwd_sm100.cu"]
 HEADERS = ["kernels.h", "ptx_sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

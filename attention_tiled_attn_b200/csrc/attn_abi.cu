@@ -203,6 +203,51 @@ int attn_fwd_streaming(const void* q, const void* k, const void* v, void* out, f
                        window, keep_first, bias, dtype, stream_ptr);
 }
 
+int attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+             float* dq, float* dk, float* dv, float* dsink, int N, int Hq, int H, int L, int S, int E, int Ev,
+             float scale, int mode, const float* sink_logits, int mask_kind, int window, void* stream_ptr) {
+  using namespace attn;
+  if (!out || !dout || !lse || !dq || !dk || !dv) return ATTN_ERR_NULL_POINTER;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_SLIDING_WINDOW) return ATTN_ERR_MASK;
+  if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window < 1) return ATTN_ERR_WINDOW;
+  int st = validate(q, k, v, dq, nullptr, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, nullptr, ATTN_BF16);
+  if (st != ATTN_OK) return st;
+  if (!aligned(out, 16) || !aligned(dout, 16) || !aligned(lse, 4) || !aligned(dq, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16) || (dsink && !aligned(dsink, 4)))
+    return ATTN_ERR_ALIGNMENT;
+  int dev = 0, sms = 0, major = 0;
+  if (device_info(&dev, &sms, &major) != ATTN_OK) return ATTN_ERR_CUDA;
+  if (major != 10) return ATTN_ERR_DEVICE;
+  BwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.dout = dout;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dsink = sink_logits ? dsink : nullptr;
+  a.sink = sink_logits;
+  a.N = N;
+  a.Hq = Hq;
+  a.H = H;
+  a.L = L;
+  a.S = S;
+  a.E = E;
+  a.Ev = Ev;
+  a.scale = scale;
+  a.rbf = (mode == ATTN_RBF);
+  a.mask_kind = mask_kind;
+  a.window = window;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  void* ws = nullptr;
+  st = ensure_workspace(dev, bwd_workspace_bytes(a), stream, &ws);
+  if (st != ATTN_OK) return st;
+  return launch_bwd_bf16(a, ws, stream);
+}
+
 int attn_fwd_padded(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L,
                     int S, int E, int Ev, float scale, int mode, const float* sink_logits, int mask_kind, int window,
                     const unsigned int* mask_bits, const int* kv_start, const int* kv_end, int dtype,
@@ -287,8 +332,9 @@ int attn_device_status(void* stream_ptr) {
   cudaStream_t s = static_cast<cudaStream_t>(stream_ptr);
   const unsigned int a = take_status_prefill(s);
   const unsigned int b = take_status_decode(s);
-  if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu) return ATTN_ERR_CUDA;
-  return (a | b) ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
+  const unsigned int c = take_status_bwd(s);
+  if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu) return ATTN_ERR_CUDA;
+  return (a | b | c) ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
 }
 
 int attn_version(void) { return 10000; }

@@ -59,6 +59,28 @@ bool make_map_rows(void* map, const void* base, int dim, long long rows, long lo
 int launch_exp2_poly_eval(const float* x, float* y, int n, cudaStream_t stream);
 
 // Read-and-clear of each kernel file's device fault word (synchronises `s`).
+// Backward (bf16): validated arguments of one attn_bwd call.
+struct BwdArgs {
+  const void* q;       // [N, Hq, L, E] bf16
+  const void* k;       // [N, H, S, E]
+  const void* v;       // [N, H, S, Ev]
+  const void* out;     // [N, Hq, L, Ev] forward output
+  const void* dout;    // [N, Hq, L, Ev] gradient of the loss with respect to out
+  const float* lse;    // [N, Hq, L] forward lse (natural log, sink included)
+  float* dq;           // [N, Hq, L, E]
+  float* dk;           // [N, H, S, E]
+  float* dv;           // [N, H, S, Ev]
+  float* dsink;        // [Hq] or nullptr
+  const float* sink;   // [Hq] or nullptr
+  int N, Hq, H, L, S, E, Ev;
+  float scale;
+  bool rbf;
+  int mask_kind, window;
+};
+size_t bwd_workspace_bytes(const BwdArgs& a);
+int launch_bwd_bf16(const BwdArgs& a, void* workspace, cudaStream_t stream);
+unsigned int take_status_bwd(cudaStream_t s);
+
 unsigned int take_status_prefill(cudaStream_t s);
 unsigned int take_status_decode(cudaStream_t s);
 

@@ -127,6 +127,9 @@ def work_units(r: sw.Recipe):
     if is_decode(r):
         kv_bytes = r.N * r.H * decode_keys(r) * (r.E + r.Ev) * 2
         return kv_bytes, "GB/s", "hbm"
+    if r.backward:
+        # S^T, dP^T, dV, dK and dQ products: 2 (3E + 2Ev) flops per visible pair
+        return 2 * (3 * r.E + 2 * r.Ev) * visible_pairs_total(r) * r.Hq, "TFLOP/s", "tensor"
     flops = 2 * (r.E + r.Ev) * visible_pairs_total(r) * r.Hq
     return flops, "TFLOP/s", "tensor"
 
@@ -272,7 +275,18 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
     lse = torch.empty((r.N, r.Hq, r.L), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
+    if r.backward:
+        # the forward's output and lse, and a seeded dout, are inputs of the timed backward
+        attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=r.mode, sink=t["sink"], mask_kind=r.mask_kind,
+                      window=r.window, out=out, lse=lse, stream=stream)
+        dout = torch.empty_like(out)
+        sgpu.normal_into(dout, sw.stream_key(r.seed, sw.STREAM_DOUT))
+
     def step():
+        if r.backward:
+            attn.attn_bwd(t["q"], t["k"], t["v"], out, lse, dout, scale=r.scale, mode=r.mode, sink=t["sink"],
+                          mask_kind=r.mask_kind, window=r.window, stream=stream)
+            return
         if r.n_sel > 0:
             attn.attn_decode_indexed(t["q"], t["k"], t["v"], t["key_idx"], scale=r.scale, sink=t["sink"],
                                      mask_kind=r.mask_kind, window=r.window, bias=t["bias"], out=out, lse=lse,
@@ -475,12 +489,14 @@ def ours(args):
             runs.append((args.workload + ":keep_bits_random10", dataclasses.replace(base, keep_mask="random10")))
             runs.append((args.workload + ":bias_random10", dataclasses.replace(base, bias="random10")))
             runs.append((args.workload + ":left_pad_upto50", dataclasses.replace(base, pad_left=0.5)))
+            runs.append((args.workload + ":backward", dataclasses.replace(base, backward=True)))
         for name in names:
             r0 = sw.RECIPES[name]
             runs.append((name, r0))
             # controls for the "RBF / sink within 10% of plain dot" comparison: same shapes and data
             if r0.mode == "rbf":
                 runs.append((name + ":dot_control", dataclasses.replace(r0, mode="dot")))
+                runs.append((name + ":backward", dataclasses.replace(r0, backward=True)))
             if r0.sink != "none":
                 runs.append((name + ":no_sink_control", dataclasses.replace(r0, sink="none")))
             # StreamingLLM variant: 4 kept initial tokens plus the window (decode: a 4096-key window)

@@ -127,6 +127,36 @@ int attn_fwd_streaming(const void* q, const void* k, const void* v, void* out, f
                        int dtype, void* stream);
 
 /*
+ * attn_bwd -- gradients of attn_fwd's output with respect to q, k, v and the
+ * sink logits (bf16 inputs, fp32 gradients).  The sinks and register tokens
+ * the pages describe are learned (page "Attention Sink" sections 4.2 and 5;
+ * page "Dot-Product Attention을 거리 기반 RBF-Attention으로 교체한 실험기"
+ * trains the RBF model), so training needs these.  With P_ij = e^{z_ij - lse_i}
+ * on visible keys, D_i = dout_i . out_i and dS_ij = P_ij (dout_i . v_j - D_i):
+ *   dv_j = sum_i P_ij dout_i        dq_i = c sum_j dS_ij k_j
+ *   dk_j = c sum_i dS_ij q_i  (rbf: minus c k_j sum_i dS_ij)
+ *   dsink_h = -sum_{n,i} e^{s_h - lse_i} D_i
+ * with c = scale (dot) or 2 scale (rbf).  GQA: dk and dv sum over the query
+ * heads of each KV group.
+ *
+ *   q, k, v     the forward's inputs (bf16, attn_fwd's layouts)
+ *   out, lse    the forward's output (bf16 [N, Hq, L, Ev]) and lse (float [N, Hq, L])
+ *   dout        bf16 [N, Hq, L, Ev], the loss gradient with respect to out
+ *   dq, dk, dv  float outputs, the layouts of q, k, v (caller-owned, overwritten)
+ *   dsink       float [Hq] output, or NULL; written when sink_logits is given
+ *   scale, mode, sink_logits, mask_kind (NONE, CAUSAL, SLIDING_WINDOW), window:
+ *               as in the forward call that produced out and lse
+ * Biases, keep bits, padding and the streaming mask have no backward here.
+ * Errors: attn_fwd's codes (ATTN_ERR_NULL_POINTER also for out, dout, lse, dq,
+ * dk, dv).  Uses and grows the library workspace (N*Hq*L floats), so it is
+ * ordered with decode calls like they are with each other; no host sync.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+             const float* lse, float* dq, float* dk, float* dv, float* dsink,
+             int N, int Hq, int H, int L, int S, int E, int Ev, float scale, int mode,
+             const float* sink_logits, int mask_kind, int window, void* stream);
+
+/*
  * attn_fwd_padded -- attn_fwd with a packed boolean keep mask and per-batch key
  * padding in place of the float bias (page "SDPA란 무엇인가" §1: B holds 0 or
  * -inf; §4 trap 1: in a boolean attn_mask, True marks a pair that takes part;

@@ -50,6 +50,7 @@ STREAM_BIAS = 5
 STREAM_KEY_FACTOR = 6
 STREAM_KEY_INDEX = 7
 STREAM_PAD = 8
+STREAM_DOUT = 9
 
 LN2 = 0.6931471805599453          # double nearest ln 2
 HALF_PI = 1.5707963267948966      # double nearest pi/2
@@ -231,6 +232,7 @@ class Recipe:
     keep_mask: str = "none"   # "random10": boolean keep mask, False where the random10 bias is -inf
     pad_left: float = 0.0     # per-batch left padding: kv_start[n] = floor(u * pad_left * S)
     pad_right: float = 0.0    # per-batch right padding: kv_end[n] = S - floor(u * pad_right * S)
+    backward: bool = False    # the measured step is the backward pass (dout: N(0,1) draws of its own stream)
     sink: str = "none"    # "none", "fixed", "normal"
     sink_values: tuple = ()
     bias: str = "none"    # "none" or "random10"

@@ -1,0 +1,129 @@
+"""Backward (attn_bwd) on the GPU against the float64 oracle's attention_backward.
+
+Inputs are the seeded bf16 draws of synth.workloads; the oracle widens the same
+bits to float64 and runs its own forward, so it shares nothing with the CUDA
+path but the inputs.  dout is a second seeded bf16 draw.
+
+Tolerance (bf16 operands, fp32 accumulation): the kernel rounds P and dS to bf16
+before the tensor-core products (relative error 2^-9 each) and reads D from the
+bf16 forward output (2^-9); each gradient element sums O(S) or O(L) such terms
+of mixed sign, so its error is a few 2^-9 relative to the gradient's scale.
+The bar is a relative L2 error <= 2e-2 per gradient tensor and a max abs error
+<= 3e-2 * max |reference| per tensor.
+"""
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import attention_tiled_attn_b200 as attn
+from oracle import attention as orc
+from synth import gpu as sgpu
+from synth import workloads as sw
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 2e-2
+MAX_ABS_FRAC = 3e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda_ready():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from attention_tiled_attn_b200 import build as b
+    b.build()
+    sgpu.build()
+    yield
+    assert attn.device_status() == 0, "a kernel recorded a bounded-wait timeout"
+
+
+def R(name, **kw):
+    base = dict(N=1, Hq=2, H=2, L=64, S=64, E=64, Ev=64, dtype="bf16", mode="dot", scale=0.125,
+                mask_kind="none", window=0, sink="none", bias="none", seed=200)
+    base.update(kw)
+    return sw.Recipe(name, **base)
+
+
+CASES = [
+    R("b_dot_causal_300_e128_g2", L=300, S=300, E=128, Ev=128, Hq=4, H=2, mask_kind="causal"),
+    R("b_rbf_causal_257_sink", L=257, S=257, mode="rbf", mask_kind="causal", sink="fixed", sink_values=(0.0, 1.0)),
+    R("b_dot_window100_515_g3_sink", L=515, S=515, Ev=128, Hq=6, H=2, mask_kind="window", window=100,
+      sink="normal"),
+    R("b_dot_none_L200_S600_g4_e128_ev64", L=200, S=600, E=128, Ev=64, Hq=8, H=2),
+    R("b_dot_causal_L1_S1000_g4_decode", L=1, S=1000, E=128, Ev=128, Hq=8, H=2, mask_kind="causal", sink="normal",
+      scale=0.0884),
+    R("b_rbf_window64_L130_S700_e64_ev128", L=130, S=700, Ev=128, mode="rbf", mask_kind="window", window=64,
+      scale=0.05),
+    R("b_rbf_registers_260", L=260, S=260, mode="rbf", mask_kind="causal", registers=4, key_lognormal=True,
+      sinusoid_pe=True, sink="normal"),
+    R("b_dot_causal_33_g16", L=33, S=33, Hq=16, H=1, mask_kind="causal"),
+    R("b_dot_none_600_n2", L=600, S=600, N=2, E=128, Ev=128, Hq=2, H=1, sink="normal", scale=0.0884),
+]
+
+
+def _dout(r, seed=77):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((r.N, r.Hq, r.L, r.Ev))
+    return sw.bf16_round_bits(x)
+
+
+def _check(name, got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    nrm = np.linalg.norm(ref)
+    err = np.abs(got - ref)
+    scale = max(np.abs(ref).max(), 1e-30)
+    if nrm > 0:
+        rel = np.linalg.norm(got - ref) / nrm
+        assert rel <= REL_L2, f"{name}: rel L2 {rel:.3e}"
+    assert err.max() <= MAX_ABS_FRAC * scale, f"{name}: max abs {err.max():.3e} vs scale {scale:.3e}"
+    return float(err.max() / scale)
+
+
+def run_case(r):
+    host = sw.generate(r)
+    t = {x: sgpu.to_device(host[x], r) for x in ("q", "k", "v")}
+    sink = None if host["sink"] is None else torch.from_numpy(host["sink"]).cuda()
+    out, lse = attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=r.mode, sink=sink, mask_kind=r.mask_kind,
+                             window=r.window)
+    dout_bits = _dout(r)
+    dout = sgpu.to_device(dout_bits, r)
+    dq, dk, dv, dsink = attn.attn_bwd(t["q"], t["k"], t["v"], out, lse, dout, scale=r.scale, mode=r.mode, sink=sink,
+                                      mask_kind=r.mask_kind, window=r.window)
+    torch.cuda.synchronize()
+    q64, k64, v64 = (sw.as_f64(r, host[x]) for x in ("q", "k", "v"))
+    rq, rk, rv, rs = orc.attention_backward(q64, k64, v64, sw.bf16_bits_to_f64(dout_bits), scale=r.scale,
+                                            mode=r.mode,
+                                            sink=None if host["sink"] is None else host["sink"].astype(np.float64),
+                                            mask_kind=r.mask_kind, window=r.window)
+    res = {
+        "dq": _check(f"{r.name} dq", dq.cpu().numpy(), rq),
+        "dk": _check(f"{r.name} dk", dk.cpu().numpy(), rk),
+        "dv": _check(f"{r.name} dv", dv.cpu().numpy(), rv),
+    }
+    if sink is not None:
+        res["dsink"] = _check(f"{r.name} dsink", dsink.cpu().numpy(), rs)
+    else:
+        assert dsink is None
+    return res
+
+
+@pytest.mark.parametrize("r", CASES, ids=lambda r: r.name)
+def test_backward_matches_oracle(r):
+    run_case(r)
+
+
+def test_backward_repeat_calls_are_deterministic_up_to_dq_order():
+    """dk, dv and dsink are written once per key tile and are bit-identical across
+    calls; dq sums tiles in an unordered way and agrees to float32 rounding."""
+    r = dataclasses.replace(CASES[0], name="det")
+    host = sw.generate(r)
+    t = {x: sgpu.to_device(host[x], r) for x in ("q", "k", "v")}
+    out, lse = attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mask_kind=r.mask_kind)
+    dout = sgpu.to_device(_dout(r), r)
+    a = attn.attn_bwd(t["q"], t["k"], t["v"], out, lse, dout, scale=r.scale, mask_kind=r.mask_kind)
+    b = attn.attn_bwd(t["q"], t["k"], t["v"], out, lse, dout, scale=r.scale, mask_kind=r.mask_kind)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert torch.allclose(a[0], b[0], rtol=1e-5, atol=1e-6)

@@ -83,12 +83,12 @@ struct BCfg {
 };
 
 struct BwdParams {
-  const float* lse;    // [N*Hq*L] natural-log lse of the forward
-  const float* dsum;   // [N*Hq*L] D = dout . out
+  const float* lse2;   // [N*Hq*Lp] the forward's lse * log2e, -inf past L (Lp = L rounded up to 128)
+  const float* dsum;   // [N*Hq*Lp] D = dout . out, 0 past L
   float* dq;           // [N*Hq*L*E], accumulated (zeroed by the launcher)
   float* dk;           // [N*H*S*E]
   float* dv;           // [N*H*S*Ev]
-  int N, Hq, H, L, S, group;
+  int N, Hq, H, L, S, group, Lp;
   int mask_kind, window;
   int rbf;
   float c_z;           // base-2 logit per unit of q.k: scale*log2e (dot) or 2*scale*log2e (rbf)
@@ -140,9 +140,11 @@ __global__ void __launch_bounds__(BTHREADS, 1)
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8u * i; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_kt = (p.S + TB - 1) / TB;
-  const int kt = blockIdx.x % n_kt;
-  const int nh = blockIdx.x / n_kt;  // n * H + kvh
+  // key-tile-major numbering: under a causal mask the early key tiles see the most
+  // query tiles, so the heaviest CTAs are launched first
+  const int nh_total = p.N * p.H;
+  const int kt = blockIdx.x / nh_total;
+  const int nh = blockIdx.x % nh_total;  // n * H + kvh
   const int n = nh / p.H, kvh = nh % p.H;
   const int k0 = kt * TB;
   int qt_lo, qt_hi;
@@ -290,6 +292,7 @@ __global__ void __launch_bounds__(BTHREADS, 1)
       const int hq = kvh * p.group + it / n_qt;
       const int q0 = (qt_lo + it % n_qt) * TB;
       const size_t rowbase = (static_cast<size_t>(n) * p.Hq + hq) * p.L;
+      const size_t padbase = (static_cast<size_t>(n) * p.Hq + hq) * p.Lp + q0;  // 16-byte aligned
       if (!__all_sync(0xffffffffu, bwait(bar(C::B_SFULL), it & 1, abort_flag))) {
         ok = false;
         break;
@@ -301,6 +304,13 @@ __global__ void __launch_bounds__(BTHREADS, 1)
       const int ds_unit = (t & 63) >> 3;
 #pragma unroll 1
       for (int ch = 0; ch < TB / 32; ++ch) {
+        // the chunk's lse2 and D (every thread reads the same 256 bytes: L1 broadcast), issued first
+        float4 l4[8], d4[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          l4[u] = __ldg(reinterpret_cast<const float4*>(p.lse2 + padbase + ch * 32) + u);
+          d4[u] = __ldg(reinterpret_cast<const float4*>(p.dsum + padbase + ch * 32) + u);
+        }
         uint32_t sr[32], dr[32];
         tmem_ld32(tmem + lane_base + C::T_S + ch * 32, sr);
         tmem_ld32(tmem + lane_base + C::T_DP + ch * 32, dr);
@@ -311,10 +321,10 @@ __global__ void __launch_bounds__(BTHREADS, 1)
         for (int e = 0; e < 32; ++e) {
           const int c = ch * 32 + e;
           const int i = q0 + c;
-          // the query's lse (base 2) and D: every thread reads the same words (L1 broadcast)
-          const float l2 = i < p.L ? __ldg(p.lse + rowbase + i) * LOG2E : -INFINITY;
-          const float dd = i < p.L ? __ldg(p.dsum + rowbase + i) : 0.f;
-          bool vis = key_ok && i < p.L && l2 != -INFINITY;
+          const float4 lv = l4[e >> 2], dv4 = d4[e >> 2];
+          const float l2 = (e & 3) == 0 ? lv.x : (e & 3) == 1 ? lv.y : (e & 3) == 2 ? lv.z : lv.w;
+          const float dd = (e & 3) == 0 ? dv4.x : (e & 3) == 1 ? dv4.y : (e & 3) == 2 ? dv4.z : dv4.w;
+          bool vis = key_ok && l2 != -INFINITY;  // -inf past L and on rows that see no key
           if (p.mask_kind != MASK_NONE) vis = vis && j <= i + off;
           if (p.mask_kind == MASK_WINDOW) vis = vis && (i + off - j) < p.window;
           const float z2 = fmaf(__uint_as_float(sr[e]), p.c_z, -kn2);
@@ -435,17 +445,29 @@ __global__ void __launch_bounds__(BTHREADS, 1)
   }
 }
 
-// D_i = dout_i . out_i (fp32) and the sink gradient -sum_i 2^(s2 - lse2_i) D_i.
-// One warp per query row.
+// D_i = dout_i . out_i (fp32), lse2_i = lse_i * log2e, both padded per head to Lp
+// rows (D = 0, lse2 = -inf past L), and the sink gradient -sum_i 2^(s2 - lse2_i) D_i.
+// One warp per padded row.
 template <int EV>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ out,
                                                       const __nv_bfloat16* __restrict__ dout,
                                                       const float* __restrict__ lse, const float* __restrict__ sink,
-                                                      float* __restrict__ dsum, float* __restrict__ dsink, int Hq,
-                                                      int L, long long rows) {
-  const long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+                                                      float* __restrict__ dsum, float* __restrict__ lse2,
+                                                      float* __restrict__ dsink, int Hq, int L, int Lp,
+                                                      long long prows) {
+  const long long pr = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
+  if (pr >= prows) return;
+  const long long head = pr / Lp;
+  const int i = static_cast<int>(pr % Lp);
+  if (i >= L) {
+    if (lane == 0) {
+      dsum[pr] = 0.f;
+      lse2[pr] = -INFINITY;
+    }
+    return;
+  }
+  const long long r = head * L + i;
   float acc = 0.f;
   for (int e = lane * 2; e < EV; e += 64) {
     const __nv_bfloat162 o2 = *reinterpret_cast<const __nv_bfloat162*>(out + r * EV + e);
@@ -456,25 +478,30 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (lane == 0) {
-    dsum[r] = acc;
+    const float l = lse[r];
+    dsum[pr] = acc;
+    lse2[pr] = l * LOG2E;
     if (sink != nullptr) {
-      const int hq = static_cast<int>((r / L) % Hq);
-      const float l = lse[r];
+      const int hq = static_cast<int>(head % Hq);
       if (l != -INFINITY) atomicAdd(dsink + hq, -ex2((sink[hq] - l) * LOG2E) * acc);
     }
   }
 }
 
 template <int E, int EV>
-int launch_bwd_impl(const BwdArgs& a, float* dsum, cudaStream_t stream) {
+int launch_bwd_impl(const BwdArgs& a, float* ws, cudaStream_t stream) {
   using C = BCfg<E, EV>;
   const long long rows = static_cast<long long>(a.N) * a.Hq * a.L;
+  const int Lp = (a.L + TB - 1) / TB * TB;
+  const long long prows = static_cast<long long>(a.N) * a.Hq * Lp;
+  float* dsum = ws;
+  float* lse2 = ws + prows;
   if (cudaMemsetAsync(a.dq, 0, static_cast<size_t>(rows) * E * sizeof(float), stream) != cudaSuccess) return -13;
   if (a.dsink && cudaMemsetAsync(a.dsink, 0, static_cast<size_t>(a.Hq) * sizeof(float), stream) != cudaSuccess)
     return -13;
-  bwd_pre_kernel<EV><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.out), static_cast<const __nv_bfloat16*>(a.dout), a.lse, a.sink, dsum,
-      a.dsink, a.Hq, a.L, rows);
+  bwd_pre_kernel<EV><<<static_cast<unsigned>((prows + 7) / 8), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(a.out), static_cast<const __nv_bfloat16*>(a.dout), a.lse, a.sink, dsum, lse2,
+      a.dsink, a.Hq, a.L, Lp, prows);
   if (cudaGetLastError() != cudaSuccess) return -13;
   CUtensorMap tq, tk, tv, tdo;
   if (!make_map_rows(&tq, a.q, E, a.L, static_cast<long long>(a.N) * a.Hq, TB)) return -13;
@@ -482,8 +509,9 @@ int launch_bwd_impl(const BwdArgs& a, float* dsum, cudaStream_t stream) {
   if (!make_map_rows(&tk, a.k, E, a.S, static_cast<long long>(a.N) * a.H, TB)) return -13;
   if (!make_map_rows(&tv, a.v, EV, a.S, static_cast<long long>(a.N) * a.H, TB)) return -13;
   BwdParams p{};
-  p.lse = a.lse;
+  p.lse2 = lse2;
   p.dsum = dsum;
+  p.Lp = Lp;
   p.dq = a.dq;
   p.dk = a.dk;
   p.dv = a.dv;
@@ -513,7 +541,8 @@ int launch_bwd_impl(const BwdArgs& a, float* dsum, cudaStream_t stream) {
 unsigned int take_status_bwd(cudaStream_t s) { return take_device_status_local(s); }
 
 size_t bwd_workspace_bytes(const BwdArgs& a) {
-  return static_cast<size_t>(a.N) * a.Hq * a.L * sizeof(float);
+  const size_t Lp = (static_cast<size_t>(a.L) + TB - 1) / TB * TB;
+  return 2 * static_cast<size_t>(a.N) * a.Hq * Lp * sizeof(float);  // D and lse2, padded per head
 }
 
 int launch_bwd_bf16(const BwdArgs& a, void* workspace, cudaStream_t stream) {

@@ -326,9 +326,9 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback"},
-        "launches_per_step": 2 if is_decode(r) else 1,
+        "launches_per_step": 2 if (is_decode(r) or r.backward) else 1,  # decode: partial + combine; backward: pre + main
         "clocks": sampler.summary() if sampler else None,
-        "tensors": t, "out": out, "lse": lse,
+        "tensors": t, "out": out, "lse": lse, "dout": dout if r.backward else None,
     }
     return res
 
@@ -341,6 +341,8 @@ def e2e_measure(res, steps, warmup):
     import attention_tiled_attn_b200 as attn
     r = res["recipe"]
     t = res["tensors"]
+    if r.backward:
+        return e2e_backward(res, steps, warmup)
     names = ("q", "k", "v", "key_idx") if r.n_sel > 0 else ("q", "k", "v")
     host = {k: t[k].cpu().pin_memory() for k in names}
     dev = {k: torch.empty_like(t[k]) for k in names}
@@ -382,6 +384,48 @@ def e2e_measure(res, steps, warmup):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}, secs
 
 
+def e2e_backward(res, steps, warmup):
+    """The backward through the public API with pinned host buffers: every step copies
+    q, k, v, out, lse and dout host->device, runs attn_bwd and reads dq, dk, dv back."""
+    import torch
+
+    import attention_tiled_attn_b200 as attn
+    r = res["recipe"]
+    t = res["tensors"]
+    src = {"q": t["q"], "k": t["k"], "v": t["v"], "out": res["out"], "lse": res["lse"], "dout": res["dout"]}
+    host = {k: x.cpu().pin_memory() for k, x in src.items()}
+    dev = {k: torch.empty_like(x) for k, x in src.items()}
+    stream = torch.cuda.current_stream()
+    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    outs_host = None
+
+    def step():
+        nonlocal outs_host
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        g = attn.attn_bwd(dev["q"], dev["k"], dev["v"], dev["out"], dev["lse"], dev["dout"], scale=r.scale,
+                          mode=r.mode, sink=t["sink"], mask_kind=r.mask_kind, window=r.window, stream=stream)
+        if outs_host is None:
+            outs_host = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in g[:3]]
+        for hbuf, x in zip(outs_host, g[:3]):
+            hbuf.copy_(x, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    secs = a.elapsed_time(b) / 1e3
+    d2h = sum(x.numel() * x.element_size() for x in outs_host)
+    return {"value": round(rate(res["amount"], secs / steps, res["unit"]), 3), "unit": res["unit"],
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}, secs
+
+
 def _oracle_cores():
     try:
         from threadpoolctl import threadpool_info
@@ -411,12 +455,22 @@ class OracleSample:
 
     def rows_amount(self, rows):
         r = self.r
+        if r.backward:
+            return work_units(r)[0] / (r.N * r.Hq) * rows.size / r.L
         if r.n_sel > 0:
             return work_units(r)[0] / (r.N * r.Hq) * rows.size / r.L
         return float(row_pairs(r, rows).sum()) * self.per_pair
 
     def run(self, rows):
         r = self.r
+        if r.backward:
+            # the oracle backward of this head (all L rows; it recomputes its forward); dout: seeded draws
+            dout = np.random.default_rng(self.hq).standard_normal((1, 1, r.L, r.Ev))
+            self.orc.attention_backward(self.q[None, None], self.k[None, None], self.v[None, None], dout,
+                                        scale=r.scale, mode=r.mode,
+                                        sink=None if self.sink is None else np.array([self.sink]),
+                                        mask_kind=r.mask_kind, window=r.window)
+            return self.rows_amount(np.arange(r.L))
         if r.n_sel > 0:
             # the index-set oracle on this head's L rows (decode: L is small); rows counts the work done
             self.orc.attention_over_index_set(
@@ -447,7 +501,7 @@ def cpu_baseline(r: sw.Recipe, budget_s: float = 12.0, wall_limit_s: float = 40.
         for hq in range(r.Hq):
             smp = OracleSample(r, n, hq, key_idx)
             heads += 1
-            for i1 in range(r.L, 0, -256):
+            for i1 in (range(r.L, 0, -r.L) if r.backward else range(r.L, 0, -256)):
                 rows = np.arange(max(0, i1 - 256), i1)
                 t0 = time.perf_counter()
                 done += smp.run(rows)
@@ -623,6 +677,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch N (profiling captures of a smaller case)")
+    ap.add_argument("--backward", action="store_true",
+                    help="measure the backward pass (attn_bwd) of the workload instead of its forward")
     ap.add_argument("--select", type=int, default=None, metavar="K",
                     help="decode workloads: attend over K listed keys per KV head (attn_decode_indexed), "
                          "a random K-subset of the cache")
@@ -632,6 +688,11 @@ def main():
     import dataclasses
     if args.batch is not None:
         sw.RECIPES[args.workload] = dataclasses.replace(sw.RECIPES[args.workload], N=args.batch)
+    if args.backward:
+        rr = sw.RECIPES[args.workload]
+        if rr.dtype != "bf16" or rr.bias != "none":
+            raise SystemExit("--backward needs a bf16 workload without a bias")
+        sw.RECIPES[args.workload] = dataclasses.replace(rr, backward=True)
     if args.select is not None:
         rr = sw.RECIPES[args.workload]
         if args.select < 1 or not is_decode(rr):

@@ -55,6 +55,7 @@ NCU_TRAFFIC_BYTES = {
     "decode_sink_gqa_128k_bf16": 16 * (1_073_819_648 + 6_067_200),
     # the same kernel's gather variant over 3971 listed keys (--select 3971), batch-2 capture scaled by 16
     "decode_sink_gqa_128k_bf16:select3971": 16 * (32_867_072 + 5_376),
+    "dot_causal_2k_bf16:backward": 453_322_496 + 293_284_608,  # bwd_kernel<128,128> (--backward)
 }
 
 
@@ -319,7 +320,8 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
     else:
         peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         punit = "GB/s"
-    traffic = NCU_TRAFFIC_BYTES.get(name if r.n_sel == 0 else f"{name}:select{r.n_sel}")
+    key = name + (":backward" if r.backward else "") + (f":select{r.n_sel}" if r.n_sel > 0 else "")
+    traffic = NCU_TRAFFIC_BYTES.get(key)
     res = {
         "recipe": r, "amount": amount, "unit": unit, "secs_max": secs_max, "secs": secs,
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": punit,

@@ -583,6 +583,20 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
             continue;
           }
         }
+        // EXT: this row's keep bits for the tile, loaded before the wait for S so their latency hides
+        // behind it (words past the row's end read as 0: keys >= S are masked anyway)
+        uint32_t m0 = ~0u, m1 = ~0u, m2 = ~0u, m3 = ~0u;
+        if constexpr (EXT) {
+          if (pa.bits != nullptr && i < p.L) {
+            const int kw = (jb * BN) >> 5;
+            const uint32_t* brow = pa.bits + static_cast<size_t>(i) * pa.words + kw;
+            const int wl = pa.words - kw;
+            m0 = __ldg(brow);
+            m1 = wl > 1 ? __ldg(brow + 1) : 0u;
+            m2 = wl > 2 ? __ldg(brow + 2) : 0u;
+            m3 = wl > 3 ? __ldg(brow + 3) : 0u;
+          }
+        }
         {
           const bool ws = wait_bar(bar(C::B_SFULL + t), sc & 1, abort_flag);
           if (!__all_sync(0xffffffffu, ws)) {
@@ -649,12 +663,8 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
           }
         }
         if constexpr (EXT) {
-          // keep bits of this row's 128 keys (words past the row's end read as 0: keys >= S are masked anyway)
+          // keep bits of this row's 128 keys (loaded above)
           if (pa.bits != nullptr && i < p.L) {
-            const uint32_t* brow = pa.bits + static_cast<size_t>(i) * pa.words + (k0 >> 5);
-            const int wl = pa.words - (k0 >> 5);
-            const uint32_t m0 = __ldg(brow), m1 = wl > 1 ? __ldg(brow + 1) : 0u;
-            const uint32_t m2 = wl > 2 ? __ldg(brow + 2) : 0u, m3 = wl > 3 ? __ldg(brow + 3) : 0u;
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               if (!((m0 >> c) & 1u)) z[c] = -INFINITY;

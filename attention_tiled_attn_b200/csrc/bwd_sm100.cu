@@ -481,7 +481,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
     const float l = lse[r];
     dsum[pr] = acc;
     lse2[pr] = l * LOG2E;
-    if (sink != nullptr) {
+    if (sink != nullptr && dsink != nullptr) {  // a caller may pass sink logits without asking for dsink
       const int hq = static_cast<int>(head % Hq);
       if (l != -INFINITY) atomicAdd(dsink + hq, -ex2((sink[hq] - l) * LOG2E) * acc);
     }

@@ -127,3 +127,26 @@ def test_backward_repeat_calls_are_deterministic_up_to_dq_order():
     b = attn.attn_bwd(t["q"], t["k"], t["v"], out, lse, dout, scale=r.scale, mask_kind=r.mask_kind)
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
     assert torch.allclose(a[0], b[0], rtol=1e-5, atol=1e-6)
+
+
+def test_backward_with_sink_but_no_dsink_output():
+    """Through the C entry point: sink logits given, dsink NULL. The call succeeds, writes dq, dk, dv
+    (equal to the call that also returns dsink) and touches no dsink memory."""
+    r = dataclasses.replace(CASES[2], name="no_dsink")
+    host = sw.generate(r)
+    t = {x: sgpu.to_device(host[x], r) for x in ("q", "k", "v")}
+    sink = torch.from_numpy(host["sink"]).cuda()
+    out, lse = attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, sink=sink, mask_kind=r.mask_kind,
+                             window=r.window)
+    dout = sgpu.to_device(_dout(r), r)
+    ref = attn.attn_bwd(t["q"], t["k"], t["v"], out, lse, dout, scale=r.scale, sink=sink, mask_kind=r.mask_kind,
+                        window=r.window)
+    dq, dk, dv = (torch.empty_like(x) for x in ref[:3])
+    st = attn.attn_bwd_raw(t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), out.data_ptr(),
+                           dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), None,
+                           r.N, r.Hq, r.H, r.L, r.S, r.E, r.Ev, r.scale, 0, sink.data_ptr(), 2, r.window,
+                           torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    torch.cuda.synchronize()
+    assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2])
+    assert torch.allclose(dq, ref[0], rtol=1e-5, atol=1e-6)

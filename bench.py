@@ -49,8 +49,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # command and counters are in profiles/.  Must be reset when the kernel changes.
 NCU_TRAFFIC_BYTES = {
     "dot_causal_2k_bf16": 137_730_304 + 12_148_480,          # prefill_kernel<128,128,dot> (plain variant)
-    "sink_gqa_window_16k_bf16": 167_928_576 + 98_604_032,    # prefill_kernel<64,64,dot>
-    "rbf_registers_4k_bf16": 37_884_672 + 392_192,           # prefill_kernel<64,64,rbf>
+    "sink_gqa_window_16k_bf16": 167_920_128 + 98_100_992,    # prefill_kernel<64,64,dot>
+    "rbf_registers_4k_bf16": 37_883_136 + 205_824,           # prefill_kernel<64,64,rbf>
     # decode_partial_kernel<128,128>: batch-2 capture scaled by 16 to batch 32
     "decode_sink_gqa_128k_bf16": 16 * (1_073_894_144 + 4_284_928),
     # the same kernel's gather variant over 3971 listed keys (--select 3971), batch-2 capture scaled by 16

@@ -256,7 +256,7 @@ def sink_grad(p_sink: np.ndarray, D: np.ndarray) -> float:
 
 
 def attention_backward(q, k, v, dout, *, scale, mode="dot", sink=None, mask_kind="none", window=0, bias=None,
-                       keep=0):
+                       keep=0, mask_keep=None, kv_start=None, kv_end=None):
     """Gradients of the forward with respect to q, k, v and the sink logits.
 
     The chain rule through the definitions above, in float64 and in this order
@@ -271,8 +271,9 @@ def attention_backward(q, k, v, dout, *, scale, mode="dot", sink=None, mask_kind
             dQ_i = 2 scale sum_j dS_ij k_j,  dK_j += 2 scale (sum_i dS_ij q_i - k_j sum_i dS_ij)
       sink: the sink's share p_i = exp(s - lse_i) gives d out_i / d s = -p_i out_i,
             so dsink_h = -sum_i p_i D_i (summed over batch and rows).
-    q, k, v, dout float64 arrays as in attention_forward.  Returns dq, dk, dv
-    (shapes of q, k, v) and dsink (Hq,) (zeros without a sink).
+    q, k, v, dout float64 arrays as in attention_forward; masks and padding as
+    there.  Returns dq, dk, dv (shapes of q, k, v) and dsink (Hq,) (zeros
+    without a sink).
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -282,12 +283,16 @@ def attention_backward(q, k, v, dout, *, scale, mode="dot", sink=None, mask_kind
     H, S = k.shape[1], k.shape[2]
     g = Hq // H
     out, lse = attention_forward(q, k, v, scale=scale, mode=mode, sink=sink, mask_kind=mask_kind, window=window,
-                                 bias=bias, keep=keep)
+                                 bias=bias, keep=keep, mask_keep=mask_keep, kv_start=kv_start, kv_end=kv_end)
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     dsink = np.zeros(Hq, dtype=np.float64)
     rows = np.arange(L)
-    vis = visible(rows, S, L, mask_kind, window, keep)
+    vis_kind = visible(rows, S, L, mask_kind, window, keep)
     for n in range(N):
+        rng = None
+        if kv_start is not None or kv_end is not None:
+            rng = (0 if kv_start is None else int(kv_start[n]), S if kv_end is None else int(kv_end[n]))
+        vis = padded_visible(vis_kind, mask_keep, rng)
         for hq in range(Hq):
             kvh = hq // g
             z = logits(q[n, hq], k[n, kvh], scale, mode)

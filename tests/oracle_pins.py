@@ -528,6 +528,46 @@ def check_backward_finite_differences(seed=17):
                     assert np.all(ds == 0.0)
 
 
+def check_backward_finite_differences_masks(seed=19):
+    """The gradients under the streaming mask, and under keep bits with key padding,
+    against central differences of the forward with the same mask (GQA, a sink)."""
+    rng = np.random.default_rng(seed)
+    N, Hq, H, L, S, E, Ev = 2, 2, 1, 5, 8, 3, 2
+    h = 1e-6
+    keep_m = rng.random((L, S)) < 0.7
+    cfgs = [dict(mask_kind="streaming", window=3, keep=2),
+            dict(mask_kind="causal", mask_keep=keep_m, kv_start=np.array([1, 0]), kv_end=np.array([8, 6]))]
+    for mode in ("dot", "rbf"):
+        for cfg in cfgs:
+            q, k, v = _rand(rng, N, Hq, L, E), _rand(rng, N, H, S, E), _rand(rng, N, H, S, Ev)
+            Wt = _rand(rng, N, Hq, L, Ev)
+            sink = rng.standard_normal(Hq)
+            kw = dict(scale=0.6, mode=mode, **cfg)
+
+            def loss(q_, k_, v_, s_):
+                o, _ = orc.attention_forward(q_, k_, v_, sink=s_, **kw)
+                return float(np.sum(o * Wt))
+
+            dq, dk, dv, ds = orc.attention_backward(q, k, v, Wt, sink=sink, **kw)
+            for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+                it = np.nditer(arr, flags=["multi_index"])
+                for _ in it:
+                    idx = it.multi_index
+                    a, b = arr.copy(), arr.copy()
+                    a[idx] += h
+                    b[idx] -= h
+                    args_a = {"q": (a, k, v), "k": (q, a, v), "v": (q, k, a)}[name]
+                    args_b = {"q": (b, k, v), "k": (q, b, v), "v": (q, k, b)}[name]
+                    fd = (loss(*args_a, sink) - loss(*args_b, sink)) / (2 * h)
+                    assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (mode, cfg["mask_kind"], name, idx)
+            for hh in range(Hq):
+                sa, sb = sink.copy(), sink.copy()
+                sa[hh] += h
+                sb[hh] -= h
+                fd = (loss(q, k, v, sa) - loss(q, k, v, sb)) / (2 * h)
+                assert abs(fd - ds[hh]) <= 1e-6 * max(1.0, abs(fd)), (mode, cfg["mask_kind"], "sink")
+
+
 def check_backward_matches_sdpa_autograd(seed=18):
     """Dot mode without a sink: the gradients equal PyTorch's SDPA autograd in
     float64 (no mask, bottom-right causal, and an additive 0/-inf bias)."""
@@ -554,5 +594,5 @@ ALL_CHECKS = [
     check_zero_sink_equivalence, check_convexity, check_causal_alignment_golden,
     check_fully_masked_rows, check_window_semantics, check_permutation_equivariance,
     check_gqa_repeat, check_streaming_mask, check_index_set, check_padding_and_keep_mask,
-    check_backward_finite_differences, check_backward_matches_sdpa_autograd,
+    check_backward_finite_differences, check_backward_finite_differences_masks, check_backward_matches_sdpa_autograd,
 ]

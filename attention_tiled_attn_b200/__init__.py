@@ -54,7 +54,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_fwd_padded.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp, vp, vp, ci,
                                     vp]
     lib.attn_fwd_padded.restype = ci
-    lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp]
+    lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, ci,
+                             vp, vp, vp, vp]
     lib.attn_bwd.restype = ci
     lib.attn_status_string.argtypes = [ci]
     lib.attn_status_string.restype = ctypes.c_char_p
@@ -98,22 +99,28 @@ def attn_fwd_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, N, Hq, H, L, S, E, Ev, s
 
 
 def attn_bwd_raw(q_ptr, k_ptr, v_ptr, out_ptr, dout_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr, dsink_ptr, N, Hq, H, L, S,
-                 E, Ev, scale, mode, sink_ptr, mask_kind, window, stream_ptr) -> int:
+                 E, Ev, scale, mode, sink_ptr, mask_kind, window, stream_ptr, keep_first=0, bits_ptr=None,
+                 start_ptr=None, end_ptr=None) -> int:
     """The backward C entry point with integer pointers; returns the status code."""
     lib = load_library()
     c = lambda p: None if p is None else ctypes.c_void_p(int(p))  # noqa: E731
     return lib.attn_bwd(c(q_ptr), c(k_ptr), c(v_ptr), c(out_ptr), c(dout_ptr), c(lse_ptr), c(dq_ptr), c(dk_ptr),
                         c(dv_ptr), c(dsink_ptr), int(N), int(Hq), int(H), int(L), int(S), int(E), int(Ev),
-                        float(scale), int(mode), c(sink_ptr), int(mask_kind), int(window), c(stream_ptr))
+                        float(scale), int(mode), c(sink_ptr), int(mask_kind), int(window), int(keep_first),
+                        c(bits_ptr), c(start_ptr), c(end_ptr), c(stream_ptr))
 
 
 def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
              dout: torch.Tensor, *, scale: float, mode: str = "dot", sink: torch.Tensor | None = None,
-             mask_kind: str = "none", window: int = 0, stream: torch.cuda.Stream | None = None):
+             mask_kind: str = "none", window: int = 0, stream: torch.cuda.Stream | None = None, keep_first: int = 0,
+             mask_bits: torch.Tensor | None = None, kv_start: torch.Tensor | None = None,
+             kv_end: torch.Tensor | None = None):
     """Gradients (dq, dk, dv, dsink) of attn_fwd's output; float32 tensors, dsink None without a sink.
 
     q, k, v, out, dout: contiguous bfloat16 CUDA tensors (the forward's inputs and
     output, and the loss gradient of the output); lse: the forward's float32 lse.
+    mask_kind "streaming" with window and keep_first, and mask_bits / kv_start /
+    kv_end, mirror attn_fwd's arguments.
     """
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
         if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
@@ -134,10 +141,20 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
     dsink = torch.empty(Hq, dtype=torch.float32, device=q.device) if sink is not None else None
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
+    for name, t, shape in (("mask_bits", mask_bits, (L, (S + 31) // 32)), ("kv_start", kv_start, (N,)),
+                           ("kv_end", kv_end, (N,))):
+        if t is not None and (not t.is_cuda or t.dtype != torch.int32 or tuple(t.shape) != shape
+                              or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA int32 tensor of shape {shape}")
+    if mask_kind == "streaming":
+        kind, keep = MASKS["window"], int(keep_first)
+    else:
+        kind, keep = MASKS[mask_kind], 0
     with torch.cuda.device(q.device):
         st = load_library().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                      _ptr(dv), _ptr(dsink), N, Hq, H, L, S, E, Ev, float(scale), MODES[mode],
-                                     _ptr(sink), MASKS[mask_kind], int(window), ctypes.c_void_p(stream.cuda_stream))
+                                     _ptr(sink), kind, int(window), keep, _ptr(mask_bits), _ptr(kv_start),
+                                     _ptr(kv_end), ctypes.c_void_p(stream.cuda_stream))
     _check(st)
     return dq, dk, dv, dsink
 

@@ -205,11 +205,16 @@ int attn_fwd_streaming(const void* q, const void* k, const void* v, void* out, f
 
 int attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
              float* dq, float* dk, float* dv, float* dsink, int N, int Hq, int H, int L, int S, int E, int Ev,
-             float scale, int mode, const float* sink_logits, int mask_kind, int window, void* stream_ptr) {
+             float scale, int mode, const float* sink_logits, int mask_kind, int window, int keep_first,
+             const unsigned int* mask_bits, const int* kv_start, const int* kv_end, void* stream_ptr) {
   using namespace attn;
   if (!out || !dout || !lse || !dq || !dk || !dv) return ATTN_ERR_NULL_POINTER;
   if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_SLIDING_WINDOW) return ATTN_ERR_MASK;
   if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window < 1) return ATTN_ERR_WINDOW;
+  // kept keys (the streaming mask) go with the sliding window
+  if (keep_first < 0 || (keep_first > 0 && mask_kind != ATTN_MASK_SLIDING_WINDOW)) return ATTN_ERR_KEEP;
+  if ((mask_bits && !aligned(mask_bits, 4)) || (kv_start && !aligned(kv_start, 4)) || (kv_end && !aligned(kv_end, 4)))
+    return ATTN_ERR_ALIGNMENT;
   int st = validate(q, k, v, dq, nullptr, N, Hq, H, L, S, E, Ev, scale, mode, sink_logits, nullptr, ATTN_BF16);
   if (st != ATTN_OK) return st;
   if (!aligned(out, 16) || !aligned(dout, 16) || !aligned(lse, 4) || !aligned(dq, 16) || !aligned(dk, 16) ||
@@ -239,8 +244,12 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* out, const
   a.Ev = Ev;
   a.scale = scale;
   a.rbf = (mode == ATTN_RBF);
-  a.mask_kind = mask_kind;
+  a.mask_kind = keep_first > 0 ? MASK_STREAM : mask_kind;
   a.window = window;
+  a.keep = keep_first;
+  a.mask_bits = mask_bits;
+  a.kv_start = kv_start;
+  a.kv_end = kv_end;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   void* ws = nullptr;
   st = ensure_workspace(dev, bwd_workspace_bytes(a), stream, &ws);

@@ -90,6 +90,11 @@ struct BwdParams {
   float* dv;           // [N*H*S*Ev]
   int N, Hq, H, L, S, group, Lp;
   int mask_kind, window;
+  int keep;             // MASK_STREAM: kept initial keys
+  const uint32_t* bits;  // [L][words] keep bits, or nullptr
+  const int* kv_start;   // [N] or nullptr
+  const int* kv_end;     // [N] or nullptr
+  int words;
   int rbf;
   float c_z;           // base-2 logit per unit of q.k: scale*log2e (dot) or 2*scale*log2e (rbf)
   float c_kn;          // rbf: scale*log2e per unit of |k|^2
@@ -116,8 +121,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void query_tiles(const BwdParams& p, int k0, int& qt_lo, int& qt_hi) {
   const int off = p.S - p.L;
   int lo = 0, hi = p.L;  // query rows [lo, hi)
-  if (p.mask_kind != MASK_NONE) lo = max(0, k0 - off);                       // i' >= j
-  if (p.mask_kind == MASK_WINDOW) hi = min(p.L, k0 + TB - 1 + p.window - off);  // i' - j < W
+  if (p.mask_kind != MASK_NONE) lo = max(0, k0 - off);  // i' >= j
+  // i' - j < W, except that kept keys (streaming) stay visible to every later query
+  if (p.mask_kind == MASK_WINDOW || (p.mask_kind == MASK_STREAM && k0 >= p.keep))
+    hi = min(p.L, k0 + TB - 1 + p.window - off);
   qt_lo = lo / TB;
   qt_hi = hi > lo ? (hi + TB - 1) / TB : qt_lo;
 }
@@ -149,6 +156,10 @@ __global__ void __launch_bounds__(BTHREADS, 1)
   const int k0 = kt * TB;
   int qt_lo, qt_hi;
   query_tiles(p, k0, qt_lo, qt_hi);
+  // key padding of this batch: a key tile wholly outside [ks, ke) has zero gradients
+  const int ks = p.kv_start ? max(0, p.kv_start[n]) : 0;
+  const int ke = p.kv_end ? min(p.S, p.kv_end[n]) : p.S;
+  if (k0 + TB <= ks || k0 >= ke) qt_hi = qt_lo;
   const int n_qt = qt_hi - qt_lo;
   const int n_it = n_qt * p.group;  // (query head of the group, query tile) pairs
 
@@ -327,6 +338,11 @@ __global__ void __launch_bounds__(BTHREADS, 1)
           bool vis = key_ok && l2 != -INFINITY;  // -inf past L and on rows that see no key
           if (p.mask_kind != MASK_NONE) vis = vis && j <= i + off;
           if (p.mask_kind == MASK_WINDOW) vis = vis && (i + off - j) < p.window;
+          if (p.mask_kind == MASK_STREAM) vis = vis && (j < p.keep || (i + off - j) < p.window);
+          vis = vis && j >= ks && j < ke;
+          // keep bit (i, j): the 32 lanes of a warp hold 32 consecutive keys, one word (broadcast)
+          if (vis && p.bits != nullptr)
+            vis = (__ldg(p.bits + static_cast<size_t>(i) * p.words + (j >> 5)) >> (j & 31)) & 1u;
           const float z2 = fmaf(__uint_as_float(sr[e]), p.c_z, -kn2);
           const float pr = vis ? ex2(z2 - l2) : 0.f;
           const float ds = p.c_q * pr * (__uint_as_float(dr[e]) - dd);
@@ -523,6 +539,11 @@ int launch_bwd_impl(const BwdArgs& a, float* ws, cudaStream_t stream) {
   p.group = a.Hq / a.H;
   p.mask_kind = a.mask_kind;
   p.window = a.window;
+  p.keep = a.keep;
+  p.bits = a.mask_bits;
+  p.kv_start = a.kv_start;
+  p.kv_end = a.kv_end;
+  p.words = (a.S + 31) / 32;
   p.rbf = a.rbf ? 1 : 0;
   p.c_z = (a.rbf ? 2.f : 1.f) * a.scale * LOG2E;
   p.c_kn = a.scale * LOG2E;

@@ -76,6 +76,10 @@ struct BwdArgs {
   float scale;
   bool rbf;
   int mask_kind, window;
+  int keep;                   // MASK_STREAM: kept initial keys
+  const uint32_t* mask_bits;  // [L][ceil(S/32)] keep bits, or nullptr
+  const int* kv_start;        // [N] or nullptr
+  const int* kv_end;          // [N] or nullptr
 };
 size_t bwd_workspace_bytes(const BwdArgs& a);
 int launch_bwd_bf16(const BwdArgs& a, void* workspace, cudaStream_t stream);

@@ -67,7 +67,7 @@ typedef enum {
   ATTN_ERR_DEVICE = -15,        /* the current device is not sm_100 */
   ATTN_ERR_SCRATCH_LIMIT = -16, /* attn_decode_fwd_noalloc: the call needs more scratch than the fixed area holds */
   ATTN_ERR_NOT_DECODE = -17,    /* attn_decode_fwd_noalloc: not a decode-shaped bf16 call ((Hq/H)*L <= 16, dot) */
-  ATTN_ERR_KEEP = -18           /* attn_fwd_streaming: keep_first < 0 */
+  ATTN_ERR_KEEP = -18           /* keep_first < 0 (attn_fwd_streaming, attn_bwd), or kept keys without a window (attn_bwd) */
 } attn_status;
 
 /*
@@ -146,15 +146,22 @@ int attn_fwd_streaming(const void* q, const void* k, const void* v, void* out, f
  *   dsink       float [Hq] output, or NULL; written when sink_logits is given
  *   scale, mode, sink_logits, mask_kind (NONE, CAUSAL, SLIDING_WINDOW), window:
  *               as in the forward call that produced out and lse
- * Biases, keep bits, padding and the streaming mask have no backward here.
- * Errors: attn_fwd's codes (ATTN_ERR_NULL_POINTER also for out, dout, lse, dq,
- * dk, dv).  Uses and grows the library workspace (N*Hq*L floats), so it is
- * ordered with decode calls like they are with each other; no host sync.
+ *   keep_first  0, or with SLIDING_WINDOW the kept initial keys of the
+ *               streaming mask (the forward was attn_fwd_streaming)
+ *   mask_bits, kv_start, kv_end: the keep bits and key padding of an
+ *               attn_fwd_padded forward (each may be NULL)
+ * The float bias has no backward here.  Errors: attn_fwd's codes
+ * (ATTN_ERR_NULL_POINTER also for out, dout, lse, dq, dk, dv), ATTN_ERR_KEEP
+ * for keep_first < 0 or kept keys without SLIDING_WINDOW, ATTN_ERR_ALIGNMENT
+ * for mask_bits, kv_start or kv_end not 4-byte aligned.  Uses and grows the
+ * library workspace (2*N*Hq*ceil(L/128)*128 floats), so it is ordered with
+ * decode calls like they are with each other; no host sync.
  */
 int attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
              const float* lse, float* dq, float* dk, float* dv, float* dsink,
              int N, int Hq, int H, int L, int S, int E, int Ev, float scale, int mode,
-             const float* sink_logits, int mask_kind, int window, void* stream);
+             const float* sink_logits, int mask_kind, int window, int keep_first,
+             const unsigned int* mask_bits, const int* kv_start, const int* kv_end, void* stream);
 
 /*
  * attn_fwd_padded -- attn_fwd with a packed boolean keep mask and per-batch key

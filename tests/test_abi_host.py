@@ -135,11 +135,13 @@ def test_padded_argument_validation(lib, kw, status):
 
 def call_bwd(**kw):
     a = dict(q=P, k=P, v=P, out=P, dout=P, lse=P, dq=P, dk=P, dv=P, dsink=None, N=1, Hq=2, H=1, L=8, S=8, E=64,
-             Ev=64, scale=0.125, mode=0, sink=None, mask_kind=1, window=0, stream=None)
+             Ev=64, scale=0.125, mode=0, sink=None, mask_kind=1, window=0, stream=None, keep=0, bits=None,
+             start=None, end=None)
     a.update(kw)
     return attn.attn_bwd_raw(a["q"], a["k"], a["v"], a["out"], a["dout"], a["lse"], a["dq"], a["dk"], a["dv"],
                              a["dsink"], a["N"], a["Hq"], a["H"], a["L"], a["S"], a["E"], a["Ev"], a["scale"],
-                             a["mode"], a["sink"], a["mask_kind"], a["window"], a["stream"])
+                             a["mode"], a["sink"], a["mask_kind"], a["window"], a["stream"], a["keep"], a["bits"],
+                             a["start"], a["end"])
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -148,6 +150,8 @@ def call_bwd(**kw):
     (dict(N=0), -2), (dict(Hq=3, H=2), -3), (dict(E=96), -4), (dict(scale=0.0), -5), (dict(mode=7), -6),
     (dict(mask_kind=3), -7), (dict(mask_kind=2, window=0), -8), (dict(mode=2), -9),
     (dict(dq=P + 4), -11), (dict(dk=P + 8), -11), (dict(out=P + 2), -11), (dict(lse=P + 2), -11),
+    (dict(keep=-1), -18), (dict(keep=3, mask_kind=1), -18), (dict(keep=3, mask_kind=0), -18),
+    (dict(bits=P + 2), -11), (dict(start=P + 1), -11), (dict(end=P + 3), -11),
 ])
 def test_bwd_argument_validation(lib, kw, status):
     assert call_bwd(**kw) == status

@@ -61,6 +61,17 @@ CASES = [
       sinusoid_pe=True, sink="normal"),
     R("b_dot_causal_33_g16", L=33, S=33, Hq=16, H=1, mask_kind="causal"),
     R("b_dot_none_600_n2", L=600, S=600, N=2, E=128, Ev=128, Hq=2, H=1, sink="normal", scale=0.0884),
+    # the streaming mask, keep bits and key padding of attn_fwd_streaming / attn_fwd_padded
+    R("b_stream_w100_keep4_600_g2", L=600, S=600, Hq=4, H=2, mask_kind="streaming", window=100, keep=4,
+      sink="normal"),
+    R("b_rbf_stream_w64_keep130_400", L=400, S=400, mode="rbf", mask_kind="streaming", window=64, keep=130,
+      scale=0.05),
+    R("b_keep_bits_causal_300_e128", L=300, S=300, E=128, Ev=128, Hq=4, H=2, mask_kind="causal",
+      keep_mask="random10", sink="normal"),
+    R("b_left_pad_causal_500_n3", L=500, S=500, N=3, mask_kind="causal", pad_left=0.5),
+    R("b_rbf_window_keep_both_pads_450", L=450, S=450, N=2, mode="rbf", mask_kind="window", window=100,
+      keep_mask="random10", pad_left=0.3, pad_right=0.3, scale=0.05),
+    R("b_keep_right_pad_L200_S700", L=200, S=700, N=2, keep_mask="random10", pad_right=0.5, Ev=128),
 ]
 
 
@@ -86,18 +97,24 @@ def run_case(r):
     host = sw.generate(r)
     t = {x: sgpu.to_device(host[x], r) for x in ("q", "k", "v")}
     sink = None if host["sink"] is None else torch.from_numpy(host["sink"]).cuda()
+    km = host["keep"]
+    masks = dict(keep_first=r.keep,
+                 mask_bits=None if km is None else torch.from_numpy(sw.pack_mask_bits(km).view(np.int32)).cuda(),
+                 kv_start=None if host["kv_start"] is None else torch.from_numpy(host["kv_start"]).cuda(),
+                 kv_end=None if host["kv_end"] is None else torch.from_numpy(host["kv_end"]).cuda())
     out, lse = attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=r.mode, sink=sink, mask_kind=r.mask_kind,
-                             window=r.window)
+                             window=r.window, **masks)
     dout_bits = _dout(r)
     dout = sgpu.to_device(dout_bits, r)
     dq, dk, dv, dsink = attn.attn_bwd(t["q"], t["k"], t["v"], out, lse, dout, scale=r.scale, mode=r.mode, sink=sink,
-                                      mask_kind=r.mask_kind, window=r.window)
+                                      mask_kind=r.mask_kind, window=r.window, **masks)
     torch.cuda.synchronize()
     q64, k64, v64 = (sw.as_f64(r, host[x]) for x in ("q", "k", "v"))
     rq, rk, rv, rs = orc.attention_backward(q64, k64, v64, sw.bf16_bits_to_f64(dout_bits), scale=r.scale,
                                             mode=r.mode,
                                             sink=None if host["sink"] is None else host["sink"].astype(np.float64),
-                                            mask_kind=r.mask_kind, window=r.window)
+                                            mask_kind=r.mask_kind, window=r.window, keep=r.keep, mask_keep=km,
+                                            kv_start=host["kv_start"], kv_end=host["kv_end"])
     res = {
         "dq": _check(f"{r.name} dq", dq.cpu().numpy(), rq),
         "dk": _check(f"{r.name} dk", dk.cpu().numpy(), rk),

@@ -276,17 +276,18 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
     lse = torch.empty((r.N, r.Hq, r.L), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
+    masks = dict(keep_first=r.keep, mask_bits=t["mask_bits"], kv_start=t["kv_start"], kv_end=t["kv_end"])
     if r.backward:
         # the forward's output and lse, and a seeded dout, are inputs of the timed backward
         attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=r.mode, sink=t["sink"], mask_kind=r.mask_kind,
-                      window=r.window, out=out, lse=lse, stream=stream)
+                      window=r.window, out=out, lse=lse, stream=stream, **masks)
         dout = torch.empty_like(out)
         sgpu.normal_into(dout, sw.stream_key(r.seed, sw.STREAM_DOUT))
 
     def step():
         if r.backward:
             attn.attn_bwd(t["q"], t["k"], t["v"], out, lse, dout, scale=r.scale, mode=r.mode, sink=t["sink"],
-                          mask_kind=r.mask_kind, window=r.window, stream=stream)
+                          mask_kind=r.mask_kind, window=r.window, stream=stream, **masks)
             return
         if r.n_sel > 0:
             attn.attn_decode_indexed(t["q"], t["k"], t["v"], t["key_idx"], scale=r.scale, sink=t["sink"],
@@ -406,7 +407,8 @@ def e2e_backward(res, steps, warmup):
         for k in host:
             dev[k].copy_(host[k], non_blocking=True)
         g = attn.attn_bwd(dev["q"], dev["k"], dev["v"], dev["out"], dev["lse"], dev["dout"], scale=r.scale,
-                          mode=r.mode, sink=t["sink"], mask_kind=r.mask_kind, window=r.window, stream=stream)
+                          mode=r.mode, sink=t["sink"], mask_kind=r.mask_kind, window=r.window, stream=stream,
+                          keep_first=r.keep, mask_bits=t["mask_bits"], kv_start=t["kv_start"], kv_end=t["kv_end"])
         if outs_host is None:
             outs_host = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in g[:3]]
         for hbuf, x in zip(outs_host, g[:3]):
@@ -471,7 +473,7 @@ class OracleSample:
             self.orc.attention_backward(self.q[None, None], self.k[None, None], self.v[None, None], dout,
                                         scale=r.scale, mode=r.mode,
                                         sink=None if self.sink is None else np.array([self.sink]),
-                                        mask_kind=r.mask_kind, window=r.window)
+                                        mask_kind=r.mask_kind, window=r.window, keep=r.keep)
             return self.rows_amount(np.arange(r.L))
         if r.n_sel > 0:
             # the index-set oracle on this head's L rows (decode: L is small); rows counts the work done

@@ -118,18 +118,21 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // query tiles of head-local rows that can see some key of [k0, k0 + TB)
+template <bool MX>
 __device__ __forceinline__ void query_tiles(const BwdParams& p, int k0, int& qt_lo, int& qt_hi) {
   const int off = p.S - p.L;
   int lo = 0, hi = p.L;  // query rows [lo, hi)
   if (p.mask_kind != MASK_NONE) lo = max(0, k0 - off);  // i' >= j
   // i' - j < W, except that kept keys (streaming) stay visible to every later query
-  if (p.mask_kind == MASK_WINDOW || (p.mask_kind == MASK_STREAM && k0 >= p.keep))
+  if (p.mask_kind == MASK_WINDOW || (MX && p.mask_kind == MASK_STREAM && k0 >= p.keep))
     hi = min(p.L, k0 + TB - 1 + p.window - off);
   qt_lo = lo / TB;
   qt_hi = hi > lo ? (hi + TB - 1) / TB : qt_lo;
 }
 
-template <int E, int EV>
+// MX: the streaming mask, keep bits or key padding is in use (a separate instantiation,
+// so the plain masks keep their own register allocation)
+template <int E, int EV, bool MX>
 __global__ void __launch_bounds__(BTHREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -155,11 +158,14 @@ __global__ void __launch_bounds__(BTHREADS, 1)
   const int n = nh / p.H, kvh = nh % p.H;
   const int k0 = kt * TB;
   int qt_lo, qt_hi;
-  query_tiles(p, k0, qt_lo, qt_hi);
+  query_tiles<MX>(p, k0, qt_lo, qt_hi);
   // key padding of this batch: a key tile wholly outside [ks, ke) has zero gradients
-  const int ks = p.kv_start ? max(0, p.kv_start[n]) : 0;
-  const int ke = p.kv_end ? min(p.S, p.kv_end[n]) : p.S;
-  if (k0 + TB <= ks || k0 >= ke) qt_hi = qt_lo;
+  int ks = 0, ke = p.S;
+  if constexpr (MX) {
+    if (p.kv_start) ks = max(0, p.kv_start[n]);
+    if (p.kv_end) ke = min(p.S, p.kv_end[n]);
+    if (k0 + TB <= ks || k0 >= ke) qt_hi = qt_lo;
+  }
   const int n_qt = qt_hi - qt_lo;
   const int n_it = n_qt * p.group;  // (query head of the group, query tile) pairs
 
@@ -338,11 +344,13 @@ __global__ void __launch_bounds__(BTHREADS, 1)
           bool vis = key_ok && l2 != -INFINITY;  // -inf past L and on rows that see no key
           if (p.mask_kind != MASK_NONE) vis = vis && j <= i + off;
           if (p.mask_kind == MASK_WINDOW) vis = vis && (i + off - j) < p.window;
-          if (p.mask_kind == MASK_STREAM) vis = vis && (j < p.keep || (i + off - j) < p.window);
-          vis = vis && j >= ks && j < ke;
-          // keep bit (i, j): the 32 lanes of a warp hold 32 consecutive keys, one word (broadcast)
-          if (vis && p.bits != nullptr)
-            vis = (__ldg(p.bits + static_cast<size_t>(i) * p.words + (j >> 5)) >> (j & 31)) & 1u;
+          if constexpr (MX) {
+            if (p.mask_kind == MASK_STREAM) vis = vis && (j < p.keep || (i + off - j) < p.window);
+            vis = vis && j >= ks && j < ke;
+            // keep bit (i, j): the 32 lanes of a warp hold 32 consecutive keys, one word (broadcast)
+            if (vis && p.bits != nullptr)
+              vis = (__ldg(p.bits + static_cast<size_t>(i) * p.words + (j >> 5)) >> (j & 31)) & 1u;
+          }
           const float z2 = fmaf(__uint_as_float(sr[e]), p.c_z, -kn2);
           const float pr = vis ? ex2(z2 - l2) : 0.f;
           const float ds = p.c_q * pr * (__uint_as_float(dr[e]) - dd);
@@ -548,7 +556,8 @@ int launch_bwd_impl(const BwdArgs& a, float* ws, cudaStream_t stream) {
   p.c_z = (a.rbf ? 2.f : 1.f) * a.scale * LOG2E;
   p.c_kn = a.scale * LOG2E;
   p.c_q = (a.rbf ? 2.f : 1.f) * a.scale;
-  auto kern = bwd_kernel<E, EV>;
+  const bool mx = a.mask_kind == MASK_STREAM || a.mask_bits || a.kv_start || a.kv_end;
+  auto kern = mx ? bwd_kernel<E, EV, true> : bwd_kernel<E, EV, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return -13;
   const long long grid = static_cast<long long>(a.N) * a.H * ((a.S + TB - 1) / TB);

@@ -323,16 +323,16 @@ __device__ __forceinline__ void fma2g(float& d0, float& d1, float a0, float a1, 
 // 2^x = 2^n * p(f), n = round(x) (via the 1.5 * 2^23 rounding constant),
 // f = x - n in [-1/2, 1/2], p the degree-3 minimax polynomial with p(0) = 1
 // fitted by csrc/fit_exp2_poly.py (max relative error 1.02e-4); n is added to
-// the exponent field of p(f) as an integer.  x is clamped to >= -126, so the
-// result is never below 2^-126 (a masked -inf logit gives 1.2e-38, not 0).
+// the exponent field of p(f) as an integer.  Below x = -126 (a masked -inf
+// logit included) the result is exactly 0, as the hardware 2^x flushes it, so
+// a row that sees no key still sums to 0.
 constexpr float EXP2_C1 = 0.6932829022407532f;
 constexpr float EXP2_C2 = 0.24221095442771912f;
 constexpr float EXP2_C3 = 0.05500892922282219f;
 constexpr float ROUND_MAGIC = 12582912.0f;  // 1.5 * 2^23
 
 __device__ __forceinline__ void exp2_poly2(float& p0, float& p1, float x0, float x1) {
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
+  const bool z0 = x0 < -126.f, z1 = x1 < -126.f;  // also true for -inf; NaN below is discarded
   float t0, t1, n0, n1, f0, f1, q0, q1;
   fma2g(t0, t1, x0, x1, 1.f, 1.f, ROUND_MAGIC, ROUND_MAGIC);    // x + M: rounds x to an integer
   fma2g(n0, n1, t0, t1, 1.f, 1.f, -ROUND_MAGIC, -ROUND_MAGIC);  // n = round(x), exact
@@ -341,8 +341,8 @@ __device__ __forceinline__ void exp2_poly2(float& p0, float& p1, float x0, float
   fma2g(q0, q1, q0, q1, f0, f1, EXP2_C1, EXP2_C1);
   fma2g(q0, q1, q0, q1, f0, f1, 1.f, 1.f);
   // the low 9 bits of M's pattern are zero, so (bits(t) << 23) is n in the exponent field
-  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+  p0 = z0 ? 0.f : __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = z1 ? 0.f : __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
 // (d0, d1) += (a0, a1) on the packed two-lane fp32 path

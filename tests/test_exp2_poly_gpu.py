@@ -23,10 +23,13 @@ def test_exp2_poly_relative_error():
     assert np.all(np.isfinite(y)) and np.all(y > 0)
 
 
-def test_exp2_poly_clamps_below_minus_126():
+def test_exp2_poly_flushes_below_minus_126():
+    """2^-126 is the smallest normal float; below it (a masked -inf logit included)
+    the result is exactly 0, so a row that sees no key sums to 0."""
     x = np.array([-126.0, -126.5, -200.0, -1e30, -np.inf], dtype=np.float32)
     y = attn.exp2_poly_eval(torch.from_numpy(x).cuda()).cpu().numpy()
-    assert np.all(y == np.float32(2.0 ** -126))
+    assert y[0] == np.float32(2.0 ** -126)
+    assert np.all(y[1:] == 0.0)
 
 
 def test_exp2_poly_odd_length():

@@ -346,6 +346,39 @@ def check_gqa_repeat(seed=13):
         assert np.array_equal(a, b) and np.array_equal(la, lb)
 
 
+def check_magnitude_bullying(seed=20):
+    """Page "Dot-Product Attention을 거리 기반 RBF-Attention으로 교체한 실험기", section
+    details: under the dot product a key of large magnitude takes the softmax even
+    when it is poorly aligned, and under RBF, which scores by Euclidean distance, a
+    key's weight goes to zero as its magnitude grows.  One key (index 0) is put in a
+    random direction u with norm g*sqrt(E) among 63 keys of lognormal size.  As g
+    grows, its dot-product weight on the queries with q.u > 1 rises toward 1 and its
+    RBF weight on every query falls toward 0; no query's RBF argmax is that key."""
+    rng = np.random.default_rng(seed)
+    E, S, L = 16, 64, 256
+    q = _rand(rng, L, E)
+    k = _rand(rng, S, E) * np.exp(0.5 * _rand(rng, S, 1))
+    u = _rand(rng, E)
+    u /= np.linalg.norm(u)
+    v = _rand(rng, S, 4)
+    rows = np.arange(L)
+    aligned = q @ u > 1.0
+    assert aligned.sum() >= 20
+    dot_mass, rbf_max = [], []
+    for g in (1.0, 2.0, 4.0, 8.0):
+        kk = k.copy()
+        kk[0] = g * math.sqrt(E) * u
+        a_dot = orc.attend_rows(q, rows, kk, v, L, scale=0.25, mode="dot", return_weights=True)[2]
+        a_rbf = orc.attend_rows(q, rows, kk, v, L, scale=0.25, mode="rbf", return_weights=True)[2]
+        dot_mass.append(a_dot[aligned, 0].mean())
+        rbf_max.append(a_rbf[:, 0].max())
+        if g >= 4.0:
+            assert not np.any(a_rbf.argmax(axis=1) == 0)
+    assert all(a < b for a, b in zip(dot_mass, dot_mass[1:])), dot_mass
+    assert all(a > b for a, b in zip(rbf_max, rbf_max[1:])), rbf_max
+    assert dot_mass[-1] > 0.95 and rbf_max[-1] < 1e-15, (dot_mass, rbf_max)
+
+
 def check_streaming_mask(seed=14):
     """StreamingLLM mask: keep = 0 is the sliding window, keep >= i'+1 is causal,
     the visible count is |{j < keep} u {i'-W < j <= i'}|, and a decode query over
@@ -593,6 +626,6 @@ ALL_CHECKS = [
     check_dot_limits, check_uniform_entropy_golden, check_sink_limit, check_sink_mass,
     check_zero_sink_equivalence, check_convexity, check_causal_alignment_golden,
     check_fully_masked_rows, check_window_semantics, check_permutation_equivariance,
-    check_gqa_repeat, check_streaming_mask, check_index_set, check_padding_and_keep_mask,
+    check_gqa_repeat, check_magnitude_bullying, check_streaming_mask, check_index_set, check_padding_and_keep_mask,
     check_backward_finite_differences, check_backward_finite_differences_masks, check_backward_matches_sdpa_autograd,
 ]

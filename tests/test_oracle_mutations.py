@@ -26,6 +26,12 @@ def _rbf_sign_flip(q_rows, k, scale, mode, key_block=512):
     return z
 
 
+def _rbf_without_key_norm(q_rows, k, scale, mode, key_block=512):
+    if mode == "rbf":  # the dot product's logit 2*scale*q.k with no -scale*||k||^2 penalty
+        return 2.0 * scale * (np.asarray(q_rows) @ np.asarray(k).T)
+    return _real_logits(q_rows, k, scale, mode, key_block)
+
+
 def _dot_scale_dropped(q_rows, k, scale, mode, key_block=512):
     if mode == "dot":
         return q_rows @ k.T
@@ -140,6 +146,8 @@ MUTATIONS = [
     ("logits", _rbf_direct_frame, pins.check_zero_sink_equivalence),
     ("logits", _rbf_direct_frame, pins.check_rbf_expansion),
     ("logits", _rbf_sign_flip, pins.check_rbf_limits),
+    ("logits", _rbf_sign_flip, pins.check_magnitude_bullying),
+    ("logits", _rbf_without_key_norm, pins.check_magnitude_bullying),
     ("logits", _dot_scale_dropped, pins.check_dot_matches_sdpa),
     ("visible", _top_left, pins.check_causal_alignment_golden),
     ("visible", _top_left, pins.check_dot_matches_sdpa),

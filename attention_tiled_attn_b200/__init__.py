@@ -84,6 +84,23 @@ def _check(status: int):
         raise AttnError(status, status_string(status))
 
 
+def _check_kinds(mode: str, mask_kind: str, keep_first: int = 0, masks=None):
+    """Rejects an unknown mode or mask kind, and kept keys without the streaming mask."""
+    if mode not in MODES:
+        raise ValueError(f"unknown mode {mode!r}")
+    if mask_kind not in (masks or (*MASKS, "streaming")):
+        raise ValueError(f"unknown mask kind {mask_kind!r}")
+    if int(keep_first) != 0 and mask_kind != "streaming":
+        raise ValueError("keep_first needs mask_kind 'streaming'")
+
+
+def _same_device(ref: torch.Tensor, **tensors):
+    """The library reads every pointer on ref's device; a tensor elsewhere is rejected."""
+    for name, t in tensors.items():
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, not on {ref.device} with q")
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -122,6 +139,7 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
     mask_kind "streaming" with window and keep_first, and mask_bits / kv_start /
     kv_end, mirror attn_fwd's arguments.
     """
+    _check_kinds(mode, mask_kind, keep_first)
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
         if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
             raise ValueError(f"{name} must be a contiguous 4-D bfloat16 CUDA tensor")
@@ -135,17 +153,19 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
     if sink is not None and (sink.dtype != torch.float32 or sink.numel() != Hq or not sink.is_cuda
                              or not sink.is_contiguous()):
         raise ValueError("sink must be a contiguous CUDA float32 tensor of Hq values")
+    for name, t, shape in (("mask_bits", mask_bits, (L, (S + 31) // 32)), ("kv_start", kv_start, (N,)),
+                           ("kv_end", kv_end, (N,))):
+        if t is not None and (not t.is_cuda or t.dtype != torch.int32 or tuple(t.shape) != shape
+                              or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA int32 tensor of shape {shape}")
+    _same_device(q, k=k, v=v, out=out, lse=lse, dout=dout, sink=sink, mask_bits=mask_bits, kv_start=kv_start,
+                 kv_end=kv_end)
     dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
     dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
     dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
     dsink = torch.empty(Hq, dtype=torch.float32, device=q.device) if sink is not None else None
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    for name, t, shape in (("mask_bits", mask_bits, (L, (S + 31) // 32)), ("kv_start", kv_start, (N,)),
-                           ("kv_end", kv_end, (N,))):
-        if t is not None and (not t.is_cuda or t.dtype != torch.int32 or tuple(t.shape) != shape
-                              or not t.is_contiguous()):
-            raise ValueError(f"{name} must be a contiguous CUDA int32 tensor of shape {shape}")
     if mask_kind == "streaming":
         kind, keep = MASKS["window"], int(keep_first)
     else:
@@ -196,8 +216,7 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float,
     word j/32 set: row may attend key j), kv_start / kv_end (N,) int32 key
     padding: any of them routes the call through attn_fwd_padded (no bias).
     """
-    if mask_kind not in MASKS and mask_kind != "streaming":
-        raise ValueError(f"unknown mask kind {mask_kind!r}")
+    _check_kinds(mode, mask_kind, keep_first)
     load_library()
     for name, t in (("q", q), ("k", k), ("v", v)):
         if not t.is_cuda:
@@ -225,6 +244,8 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float,
         raise ValueError("out has the wrong shape/dtype")
     if tuple(lse.shape) != (N, Hq, L) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse has the wrong shape/dtype")
+    _same_device(q, k=k, v=v, out=out, lse=lse, sink=sink, bias=bias, mask_bits=mask_bits, kv_start=kv_start,
+                 kv_end=kv_end)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     with torch.cuda.device(q.device):
@@ -273,6 +294,7 @@ def attn_decode_indexed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, key_i
     positions; entries outside [0, S) select nothing.  sink, bias, mask_kind
     ("none", "causal", "window") and window as in attn_fwd.
     """
+    _check_kinds("dot", mask_kind, masks=MASKS)
     for name, t in (("q", q), ("k", k), ("v", v), ("key_idx", key_idx)):
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor")
@@ -297,6 +319,11 @@ def attn_decode_indexed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, key_i
         out = torch.empty((N, Hq, L, Ev), dtype=q.dtype, device=q.device)
     if lse is None:
         lse = torch.empty((N, Hq, L), dtype=torch.float32, device=q.device)
+    if tuple(out.shape) != (N, Hq, L, Ev) or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("out has the wrong shape/dtype")
+    if tuple(lse.shape) != (N, Hq, L) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse has the wrong shape/dtype")
+    _same_device(q, k=k, v=v, key_idx=key_idx, out=out, lse=lse, sink=sink, bias=bias)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     with torch.cuda.device(q.device):

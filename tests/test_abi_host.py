@@ -162,3 +162,22 @@ def test_python_binding_rejects_cpu_tensors(lib):
     q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         attn.attn_fwd(q, q, q, scale=0.1)
+
+
+@pytest.mark.parametrize("call", [
+    lambda q: attn.attn_fwd(q, q, q, scale=0.1, mode="cosine"),
+    lambda q: attn.attn_fwd(q, q, q, scale=0.1, mask_kind="diagonal"),
+    lambda q: attn.attn_fwd(q, q, q, scale=0.1, mask_kind="causal", keep_first=4),
+    lambda q: attn.attn_fwd(q, q, q, scale=0.1, mask_kind="window", window=8, keep_first=4),
+    lambda q: attn.attn_bwd(q, q, q, q, q, q, scale=0.1, mode="cosine"),
+    lambda q: attn.attn_bwd(q, q, q, q, q, q, scale=0.1, mask_kind="window", window=8, keep_first=4),
+    lambda q: attn.attn_decode_indexed(q, q, q, q, scale=0.1, mask_kind="streaming"),
+], ids=["fwd_mode", "fwd_mask", "fwd_keep_causal", "fwd_keep_window", "bwd_mode", "bwd_keep_window",
+        "indexed_streaming"])
+def test_python_binding_rejects_unknown_kinds_and_stray_kept_keys(lib, call):
+    """Unknown mode or mask strings, and kept keys without the streaming mask, are
+    rejected before any tensor is looked at (so this holds on a host without a GPU)."""
+    import torch
+    q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="unknown mode|unknown mask kind|keep_first needs"):
+        call(q)

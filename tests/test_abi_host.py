@@ -37,6 +37,37 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, name), name
 
 
+def declared_parameters():
+    """{name: [kind of each parameter]} for every function the header declares,
+    kind one of "ptr", "float", "int" ((void) gives an empty list)."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"^\s*(?:const\s+)?\w+\**\s+\**(attn_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.M | re.S):
+        params = m.group(2).strip()
+        kinds = []
+        if params not in ("", "void"):
+            for prm in params.split(","):
+                kinds.append("ptr" if "*" in prm else "float" if re.search(r"\bfloat\b", prm) else "int")
+        out[m.group(1)] = kinds
+    return out
+
+
+def test_binding_argtypes_match_the_header(lib):
+    """Every function the binding gives argtypes takes the header's parameters, in
+    number and kind, so a changed C signature cannot be called with a stale one."""
+    decl = declared_parameters()
+    assert set(decl) == set(declared_functions())
+    kind_of = {ctypes.c_void_p: "ptr", ctypes.c_char_p: "ptr", ctypes.c_float: "float", ctypes.c_int: "int",
+               ctypes.c_uint: "int", ctypes.c_size_t: "int"}
+    checked = 0
+    for name, kinds in decl.items():
+        argtypes = getattr(getattr(lib, name), "argtypes", None)
+        if argtypes is not None:
+            assert [kind_of[a] for a in argtypes] == kinds, name
+            checked += 1
+    assert checked >= 8
+
+
 def test_status_strings(lib):
     assert attn.status_string(0) == "ok"
     for st in range(-18, 0):

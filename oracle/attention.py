@@ -52,6 +52,12 @@ in blocks of query rows so that memory stays bounded:
   the mask taken at each key's original position.  One list per (batch, KV
   head), shared by the group's query heads; entries outside [0, S) select
   nothing; a repeated entry counts once per listing.
+
+Two readings are decisions that the pages leave open.  One is the window width
+(W keys, self included).  The other is lse with a sink (ln of the full
+denominator, sink term included).  For both, parity is unpinned beyond
+internal consistency: the pins check only that each is applied the same way
+everywhere (W = 1 keeps the own key, W >= S is causal, p_sink = e^(s - lse)).
 """
 
 from __future__ import annotations

@@ -183,3 +183,19 @@ def test_gqa_head_map_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(orc, "attention_forward", forward_modulo)
     with pytest.raises(AssertionError):
         pins.check_dot_matches_sdpa()
+
+
+@pytest.mark.parametrize("dropped", ["keep", "mask_keep", "kv_start", "kv_end"])
+def test_backward_mask_argument_dropped_is_caught(monkeypatch, dropped):
+    """A backward that ignores one of the streaming mask's kept keys, the keep bits or
+    the key padding (while the forward honours it) is caught by the finite-difference
+    pin of the masked gradients."""
+    real_backward = orc.attention_backward
+
+    def backward_without(*args, **kw):
+        kw.pop(dropped, None)
+        return real_backward(*args, **kw)
+
+    monkeypatch.setattr(orc, "attention_backward", backward_without)
+    with pytest.raises(AssertionError):
+        pins.check_backward_finite_differences_masks()

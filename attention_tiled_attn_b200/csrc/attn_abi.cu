@@ -306,7 +306,7 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_MODE: return "unknown score mode";
     case ATTN_ERR_MASK: return "unknown mask kind";
     case ATTN_ERR_WINDOW: return "sliding window needs window >= 1";
-    case ATTN_ERR_KEEP: return "streaming mask needs keep_first >= 0";
+    case ATTN_ERR_KEEP: return "keep_first must be >= 0, and kept keys need the sliding window";
     case ATTN_ERR_SINK: return "ATTN_SINK needs sink logits";
     case ATTN_ERR_DTYPE: return "unknown dtype";
     case ATTN_ERR_ALIGNMENT: return "misaligned pointer (16 bytes for tensors, 4 for lse and sink)";

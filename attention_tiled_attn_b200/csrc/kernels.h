@@ -33,6 +33,11 @@ struct AttnArgs {
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
+// Checks shared by every forward entry point once it has checked its own mask
+// arguments (defined in attn_abi.cu); returns ATTN_OK or a negative status.
+int validate(const void* q, const void* k, const void* v, void* out, float* lse, int N, int Hq, int H, int L, int S,
+             int E, int Ev, float scale, int mode, const float* sink_logits, const float* bias, int dtype);
+
 // Each launcher returns 0 or a negative attn_status code.
 int launch_prefill_bf16(const AttnArgs& a, cudaStream_t stream);
 int launch_fp32(const AttnArgs& a, cudaStream_t stream);

@@ -272,14 +272,22 @@ int attn_exp2_poly_eval(const float* x, float* y, int n, void* stream);
  * Arguments, layouts, ownership and masks are those of attn_fwd (the dtype is
  * bf16).  Instead of the library's allocated workspace, the partial results
  * live in a fixed scratch array compiled into the library
- * (attn_decode_noalloc_scratch_bytes() bytes, 8 MiB, held on every GPU that
- * loads the library until the process exits).  The first call on a device
- * looks up that array's device address (cudaGetSymbolAddress) with the
- * device current; make that first call before beginning any stream capture.
+ * (attn_decode_noalloc_scratch_bytes() bytes, 8 MiB).  The array becomes
+ * resident on a device when the library's device code is loaded into that
+ * device's context: under CUDA's default lazy module loading that is the first
+ * call on the device, which therefore takes the array's 8 MiB and the code's
+ * memory once.  Make that first call during start-up, before reserving the
+ * rest of the device's memory and before beginning any stream capture (or set
+ * CUDA_MODULE_LOADING=EAGER, which loads both with the context).  The array
+ * then stays until the context is destroyed.  The first call in a context
+ * also looks up the array's device address (cudaGetSymbolAddress) with the
+ * device current; a call that finds a different context current (after
+ * cudaDeviceReset, say) looks it up again, and that call is again a first
+ * call in the sense above.
  * Calls that need more scratch than the array holds return
  * ATTN_ERR_SCRATCH_LIMIT; calls that are not decode-shaped return
- * ATTN_ERR_NOT_DECODE; neither launches anything.  The function calls no
- * cudaMalloc, cudaFree or other allocating routine.  All calls share the one
+ * ATTN_ERR_NOT_DECODE; neither launches anything.  Beyond that module load,
+ * the function calls no cudaMalloc, cudaFree or other allocating routine.  All calls share the one
  * array: calls that overlap on the GPU race and must be ordered by the
  * caller.  Nothing in the array needs clearing between calls.
  */

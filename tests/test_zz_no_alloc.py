@@ -80,6 +80,46 @@ def test_noalloc_matches_attn_fwd_twice(lib, r):
     assert attn.device_status() == 0
 
 
+def _pool_reserved_bytes(dev: int) -> int:
+    """Bytes the device's default stream-ordered pool (the one cudaMallocAsync draws on) holds."""
+    from cuda.bindings import driver as drv
+    err, pool = drv.cuDeviceGetDefaultMemPool(dev)
+    assert err == drv.CUresult.CUDA_SUCCESS, err
+    err, val = drv.cuMemPoolGetAttribute(pool, drv.CUmemPool_attribute.CU_MEMPOOL_ATTR_RESERVED_MEM_CURRENT)
+    assert err == drv.CUresult.CUDA_SUCCESS, err
+    return int(val)
+
+
+def test_noalloc_call_takes_no_device_memory(lib):
+    """With the library's own workspace released, a call after the first (which loads the
+    library's device code and the fixed array into the context) changes neither the device's
+    free memory nor what its default stream-ordered pool holds."""
+    r = CASES[0]
+    t = _inputs(r)
+    out = torch.empty((r.N, r.Hq, r.L, r.Ev), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((r.N, r.Hq, r.L), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    dev = torch.cuda.current_device()
+
+    def call():
+        st = attn.attn_decode_fwd_noalloc_raw(
+            _ptr(t["q"]), _ptr(t["k"]), _ptr(t["v"]), _ptr(out), _ptr(lse), r.N, r.Hq, r.H, r.L, r.S, r.E, r.Ev,
+            r.scale, attn.MODES[r.mode], _ptr(t["sink"]), attn.MASKS[r.mask_kind], r.window, _ptr(t["bias"]),
+            stream)
+        assert st == 0, attn.status_string(st)
+        torch.cuda.synchronize()
+
+    attn.release_workspace()
+    call()
+    free0, _ = torch.cuda.mem_get_info()
+    pool0 = _pool_reserved_bytes(dev)
+    call()
+    free1, _ = torch.cuda.mem_get_info()
+    pool1 = _pool_reserved_bytes(dev)
+    assert free1 == free0, (free0, free1)
+    assert pool1 == pool0, (pool0, pool1)
+
+
 def test_noalloc_rejects_oversized_and_non_decode_calls(lib):
     P = 0x10000  # aligned placeholder addresses: both calls are rejected before any launch
     # 2048 (batch, KV head) units of a 64-key cache need more partial slots than the fixed area holds

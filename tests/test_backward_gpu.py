@@ -7,9 +7,12 @@ path but the inputs.  dout is a second seeded bf16 draw.
 Tolerance (bf16 operands, fp32 accumulation): the kernel rounds P and dS to bf16
 before the tensor-core products (relative error 2^-9 each) and reads D from the
 bf16 forward output (2^-9); each gradient element sums O(S) or O(L) such terms
-of mixed sign, so its error is a few 2^-9 relative to the gradient's scale.
-The bar is a relative L2 error <= 2e-2 per gradient tensor and a max abs error
-<= 3e-2 * max |reference| per tensor.
+of mixed sign, so its error is a few 2^-9 (2e-3) relative to the gradient's
+scale.  Measured on a B200 over the cases below and the three full-size
+workloads, the largest errors were 4.2e-3 relative L2 and 4.3e-3 * max |ref|
+max abs for dq, dk and dv, and 1.02e-2 relative L2 for dsink (a vector of one
+sum per head, whose terms cancel).  The bar keeps about twice that: relative L2
+and max abs / max |ref| <= 1e-2 for dq, dk, dv and <= 2e-2 for dsink.
 """
 
 import dataclasses
@@ -25,8 +28,10 @@ from synth import workloads as sw
 
 pytestmark = pytest.mark.gpu
 
-REL_L2 = 2e-2
-MAX_ABS_FRAC = 3e-2
+REL_L2 = 1e-2
+MAX_ABS_FRAC = 1e-2
+DSINK_REL_L2 = 2e-2
+DSINK_MAX_ABS_FRAC = 2e-2
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -86,10 +91,12 @@ def _check(name, got, ref):
     nrm = np.linalg.norm(ref)
     err = np.abs(got - ref)
     scale = max(np.abs(ref).max(), 1e-30)
+    sink = name.endswith("dsink")
+    rel_bar, abs_bar = (DSINK_REL_L2, DSINK_MAX_ABS_FRAC) if sink else (REL_L2, MAX_ABS_FRAC)
     if nrm > 0:
         rel = np.linalg.norm(got - ref) / nrm
-        assert rel <= REL_L2, f"{name}: rel L2 {rel:.3e}"
-    assert err.max() <= MAX_ABS_FRAC * scale, f"{name}: max abs {err.max():.3e} vs scale {scale:.3e}"
+        assert rel <= rel_bar, f"{name}: rel L2 {rel:.3e}"
+    assert err.max() <= abs_bar * scale, f"{name}: max abs {err.max():.3e} vs scale {scale:.3e}"
     return float(err.max() / scale)
 
 
@@ -115,15 +122,15 @@ def run_case(r):
                                             sink=None if host["sink"] is None else host["sink"].astype(np.float64),
                                             mask_kind=r.mask_kind, window=r.window, keep=r.keep, mask_keep=km,
                                             kv_start=host["kv_start"], kv_end=host["kv_end"])
-    res = {
-        "dq": _check(f"{r.name} dq", dq.cpu().numpy(), rq),
-        "dk": _check(f"{r.name} dk", dk.cpu().numpy(), rk),
-        "dv": _check(f"{r.name} dv", dv.cpu().numpy(), rv),
-    }
+    pairs = {"dq": (dq.cpu().numpy(), rq), "dk": (dk.cpu().numpy(), rk), "dv": (dv.cpu().numpy(), rv)}
     if sink is not None:
-        res["dsink"] = _check(f"{r.name} dsink", dsink.cpu().numpy(), rs)
+        pairs["dsink"] = (dsink.cpu().numpy(), rs)
     else:
         assert dsink is None
+    res = {g: _errors(got, ref) for g, (got, ref) in pairs.items()}
+    print(f"{r.name}: " + ", ".join(f"{g} rel L2 {e[0]:.2e} max abs/max|ref| {e[1]:.2e}" for g, e in res.items()))
+    for g, (got, ref) in pairs.items():
+        _check(f"{r.name} {g}", got, ref)
     return res
 
 
@@ -167,3 +174,72 @@ def test_backward_with_sink_but_no_dsink_output():
     torch.cuda.synchronize()
     assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2])
     assert torch.allclose(dq, ref[0], rtol=1e-5, atol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# the benchmark's three backward workloads at full size
+# ---------------------------------------------------------------------------
+
+BWD_FULL = ["dot_causal_2k_bf16", "rbf_registers_4k_bf16", "sink_gqa_window_16k_bf16"]
+
+
+def _dout_slice_host(r, n, hq):
+    """dout[n, hq] as the device generator draws it for the benchmark (its own stream of the
+    counter-based generator, bf16), regenerated on the host and widened to float64."""
+    key = sw.stream_key(r.seed, sw.STREAM_DOUT)
+    x = sw.normal_f64(key, ((n * r.Hq + hq) * r.L) * r.Ev, r.L * r.Ev).reshape(r.L, r.Ev)
+    return sw.bf16_bits_to_f64(sw.bf16_round_bits(x))
+
+
+def _errors(got, ref):
+    """(relative L2 error, max abs error / max |ref|) of one gradient tensor."""
+    got = np.asarray(got, dtype=np.float64)
+    scale = max(np.abs(ref).max(), 1e-30)
+    nrm = np.linalg.norm(ref)
+    rel = float(np.linalg.norm(got - ref) / nrm) if nrm > 0 else 0.0
+    return rel, float(np.abs(got - ref).max() / scale)
+
+
+@pytest.mark.parametrize("name", BWD_FULL)
+def test_backward_full_size(name):
+    """The whole workload's backward on the GPU, in the benchmark's launch configuration
+    (forward out and lse, dout from the generator's own stream); the oracle backward of the
+    last (batch, KV head) slice -- all query heads of the group, every row and key -- gives dq
+    of those heads, dk and dv of that KV head (the last key tile and the window edge included)
+    and, with one batch, dsink of the group's heads."""
+    r = sw.RECIPES[name]
+    t = sgpu.generate_on_device(r)
+    out, lse = attn.attn_fwd(t["q"], t["k"], t["v"], scale=r.scale, mode=r.mode, sink=t["sink"],
+                             mask_kind=r.mask_kind, window=r.window)
+    dout = torch.empty_like(out)
+    sgpu.normal_into(dout, sw.stream_key(r.seed, sw.STREAM_DOUT))
+    dq, dk, dv, dsink = attn.attn_bwd(t["q"], t["k"], t["v"], out, lse, dout, scale=r.scale, mode=r.mode,
+                                      sink=t["sink"], mask_kind=r.mask_kind, window=r.window)
+    torch.cuda.synchronize()
+    assert attn.device_status() == 0
+    n, kvh = r.N - 1, r.H - 1
+    heads = list(range(kvh * r.group, (kvh + 1) * r.group))
+    got_dq = dq[n, heads].cpu().numpy()
+    got_dk = dk[n, kvh].cpu().numpy()
+    got_dv = dv[n, kvh].cpu().numpy()
+    got_ds = None if dsink is None else dsink[heads].cpu().numpy()
+    del t, out, lse, dout, dq, dk, dv, dsink
+    torch.cuda.empty_cache()
+    q = np.stack([sw.tensor_slice_f64(r, "q", n, hq) for hq in heads])[None]
+    k = sw.tensor_slice_f64(r, "k", n, kvh)[None, None]
+    v = sw.tensor_slice_f64(r, "v", n, kvh)[None, None]
+    do = np.stack([_dout_slice_host(r, n, hq) for hq in heads])[None]
+    s = sw.sink_logits(r)
+    rq, rk, rv, rs = orc.attention_backward(q, k, v, do, scale=r.scale, mode=r.mode,
+                                            sink=None if s is None else s[heads].astype(np.float64),
+                                            mask_kind=r.mask_kind, window=r.window)
+    report = {}
+    for g, (got, ref) in {"dq": (got_dq, rq[0]), "dk": (got_dk, rk[0, 0]), "dv": (got_dv, rv[0, 0])}.items():
+        report[g] = _errors(got, ref)
+        _check(f"{name} {g}", got, ref)
+    if got_ds is not None and r.N == 1:
+        # the kernel sums dsink over the batch; with one batch the slice's heads are complete
+        report["dsink"] = _errors(got_ds, rs)
+        _check(f"{name} dsink", got_ds, rs)
+    print(f"{name} backward (n={n}, kv head {kvh}): " +
+          ", ".join(f"{g} rel L2 {e[0]:.2e} max abs/max|ref| {e[1]:.2e}" for g, e in report.items()))

@@ -1,7 +1,10 @@
 """GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
 the same seeded inputs.  Small cases compare every element; the reference
-workloads run at full size in the benchmark's launch configuration and are
-compared on sampled rows."""
+workloads, and every variant of them that the benchmark times, run at full
+size in the benchmark's launch configuration and are compared on sampled
+rows."""
+
+import dataclasses
 
 import numpy as np
 import pytest
@@ -236,9 +239,9 @@ FULL = ["dot_causal_2k_bf16", "dot_bias10_2k_f32", "rbf_registers_4k_bf16", "sin
 
 def test_decode_indexed_full_size_top_k_33x():
     """The long-context decode workload (N=32, 32 query / 8 KV heads, S=131072, E=128) over a
-    33x-sparse selection (3972 keys per KV head), sampled units against the oracle."""
-    import dataclasses
-    r = dataclasses.replace(sw.RECIPES["decode_sink_gqa_128k_bf16"], name="decode_top_k_33x", n_sel=3972)
+    33x-sparse selection (3971 keys per KV head, as the benchmark times it), sampled units against
+    the oracle."""
+    r = dataclasses.replace(sw.RECIPES["decode_sink_gqa_128k_bf16"], name="decode_top_k_33x", n_sel=131072 // 33)
     t = sgpu.generate_on_device(r)
     out, lse = gu.run_gpu(r, t)
     assert torch.isfinite(out.float()).all()
@@ -251,15 +254,44 @@ def test_decode_indexed_full_size_top_k_33x():
     torch.cuda.empty_cache()
 
 
+def _variant(base: str, label: str, **kw):
+    r = dataclasses.replace(sw.RECIPES[base], name=f"{base}:{label}", **kw)
+    return pytest.param(r, id=r.name)
+
+
+# the benchmark's extra lines: controls and mask variants of the reference workloads, same shapes and data
+FULL_VARIANTS = [
+    _variant("dot_causal_2k_bf16", "steady_state_noncausal_8k", N=1, L=8192, S=8192, mask_kind="none"),
+    _variant("dot_causal_2k_bf16", "keep_bits_random10", keep_mask="random10"),
+    _variant("dot_causal_2k_bf16", "bias_random10", bias="random10"),
+    _variant("dot_causal_2k_bf16", "left_pad_upto50", pad_left=0.5),
+    _variant("rbf_registers_4k_bf16", "dot_control", mode="dot"),
+    _variant("sink_gqa_window_16k_bf16", "no_sink_control", sink="none"),
+    _variant("sink_gqa_window_16k_bf16", "streaming_keep4", mask_kind="streaming", keep=4),
+    _variant("decode_sink_gqa_128k_bf16", "no_sink_control", sink="none"),
+    _variant("decode_sink_gqa_128k_bf16", "streaming_keep4_w4096", mask_kind="streaming", window=4096, keep=4),
+]
+
+
 @pytest.mark.parametrize("name", FULL)
 def test_reference_workload_full_size(name):
-    r = sw.RECIPES[name]
+    check_full_size(sw.RECIPES[name])
+
+
+@pytest.mark.parametrize("r", FULL_VARIANTS)
+def test_bench_variant_full_size(r):
+    check_full_size(r)
+
+
+def check_full_size(r: sw.Recipe):
+    """The whole workload on the GPU; sampled rows of three (n, hq) units (two for decode) against the oracle."""
+    name = r.name
     t = sgpu.generate_on_device(r)
     out, lse = gu.run_gpu(r, t)
     assert torch.isfinite(out.float()).all()
     rng = np.random.default_rng(sum(map(ord, name)))
     units = [(0, 0), (r.N - 1, r.Hq - 1), (int(rng.integers(r.N)), int(rng.integers(r.Hq)))]
-    if name.startswith("decode"):
+    if r.L == 1:
         units = units[:2]
     for n, hq in units:
         rows = gu.sample_rows(r.L, rng, count=12 if r.L > 1 else 0)

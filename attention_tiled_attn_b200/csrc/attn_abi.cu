@@ -178,7 +178,13 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
     if (st != ATTN_OK) return st;
     return launch_decode_bf16(a, ws, need, sms, stream);
   }
-  return launch_prefill_bf16(a, stream);
+  void* ws = nullptr;
+  const size_t need = prefill_workspace_bytes(a);
+  if (need > 0) {
+    const int st2 = ensure_workspace(dev, need, stream, &ws);
+    if (st2 != ATTN_OK) return st2;
+  }
+  return launch_prefill_bf16(a, ws, need, stream);
 }
 
 }  // namespace attn

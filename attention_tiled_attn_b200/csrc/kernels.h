@@ -39,7 +39,10 @@ int validate(const void* q, const void* k, const void* v, void* out, float* lse,
              int E, int Ev, float scale, int mode, const float* sink_logits, const float* bias, int dtype);
 
 // Each launcher returns 0 or a negative attn_status code.
-int launch_prefill_bf16(const AttnArgs& a, cudaStream_t stream);
+// bf16 prefill.  A float bias (outside the streaming mask) is first turned into keep
+// bits in `ws` (prefill_workspace_bytes(a) bytes, 0 when none is needed).
+size_t prefill_workspace_bytes(const AttnArgs& a);
+int launch_prefill_bf16(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream);
 int launch_fp32(const AttnArgs& a, cudaStream_t stream);
 
 // Decode (bf16, (Hq/H) * L <= 16): key-split partial kernel + combine kernel.

@@ -95,11 +95,13 @@ struct Cfg {
   static constexpr int THREADS = NUM_WARPS * 32;
   // Register split after launch (setmaxnreg): the softmax warpgroups grow to
   // REG_SOFTMAX, the producer / issuer / key-norm warpgroup shrinks to
-  // REG_OTHER.  256 * 216 + 128 * 72 = 168 * 384, the launch budget; the host
+  // REG_OTHER.  256 * 208 + 128 * 88 = 168 * 384, the launch budget; the host
   // refuses to launch if the compiled count is lower (the .inc would never
-  // be satisfied).
-  static constexpr uint32_t REG_SOFTMAX = 216;
-  static constexpr uint32_t REG_OTHER = 72;
+  // be satisfied).  At 88 registers the producer and issuer do not spill; that
+  // took 4.5% off the causal 2k workload's cycles against a 216 / 72 split.
+  static constexpr uint32_t REG_SOFTMAX = 208;
+  static constexpr uint32_t REG_OTHER = 88;
+  static_assert(256 * REG_SOFTMAX + 128 * REG_OTHER == 168 * THREADS, "register split");
   static constexpr uint32_t TMEM_COLS = 512;
   // Pairs of each 16-pair (32-key) chunk whose exponential runs on the FMA pipe
   // (exp2_poly2) instead of the MUFU unit (16 exponentials per clock per SM).
@@ -126,6 +128,11 @@ struct PadArgs {
   const int* kv_start;   // [N] first non-padding key, or nullptr (0)
   const int* kv_end;     // [N] one past the last non-padding key, or nullptr (S)
   int words;             // ceil(S / 32)
+  // A float bias given as keep bits (bias_bits_kernel): bits hold "entry == 0", and
+  // general[i * n_kt + jb] is 1 where row i's key tile jb has an entry that is neither
+  // 0 nor -inf; such tiles add the bias itself.  nullptr without a bias.
+  const uint8_t* general;
+  int n_kt;              // ceil(S / 128)
 };
 
 // Key-tile range of a query tile; with the streaming mask also the first tile
@@ -538,7 +545,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t t_s = tmem + lane_base + t * 128;
     const uint32_t t_o = tmem + lane_base + 256 + t * EV;
-    const bool has_bias = !EXT && p.bias != nullptr;  // the EXT entry takes keep bits instead
+    const bool has_bias = p.bias != nullptr;  // EXT: only on tiles the bias pre-pass flagged as general
     const int off = p.S - p.L;
     uint32_t gk = 0;   // union key tiles seen (key-norm ring)
     uint32_t sc = 0;   // S tiles consumed (s_full / p_full phases)
@@ -586,8 +593,11 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
         // EXT: this row's keep bits for the tile, loaded before the wait for S so their latency hides
         // behind it (words past the row's end read as 0: keys >= S are masked anyway)
         uint32_t m0 = ~0u, m1 = ~0u, m2 = ~0u, m3 = ~0u;
+        bool general = !EXT;  // the float bias is added as values (EXT: only on flagged tiles)
         if constexpr (EXT) {
-          if (pa.bits != nullptr && i < p.L) {
+          if (pa.general != nullptr && i < p.L)
+            general = __ldg(pa.general + static_cast<size_t>(i) * pa.n_kt + jb) != 0;
+          if (pa.bits != nullptr && i < p.L && !general) {
             const int kw = (jb * BN) >> 5;
             const uint32_t* brow = pa.bits + static_cast<size_t>(i) * pa.words + kw;
             const int wl = pa.words - kw;
@@ -664,7 +674,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
         }
         if constexpr (EXT) {
           // keep bits of this row's 128 keys (loaded above)
-          if (pa.bits != nullptr && i < p.L) {
+          if (pa.bits != nullptr && i < p.L && !general) {
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               if (!((m0 >> c) & 1u)) z[c] = -INFINITY;
@@ -674,7 +684,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
             }
           }
         }
-        if (has_bias && bias_row != nullptr) {
+        if (has_bias && bias_row != nullptr && general) {
           const int lim = p.S - k0;
 #pragma unroll
           for (int c = 0; c < BN; ++c)
@@ -811,7 +821,7 @@ __global__ void __launch_bounds__(Cfg<E, EV, RBF>::THREADS, 1)
 // host side
 // ---------------------------------------------------------------------------
 template <int E, int EV, bool RBF, bool STREAM, bool EXT>
-int launch_impl(const AttnArgs& a, cudaStream_t stream) {
+int launch_impl(const AttnArgs& a, const uint8_t* general, cudaStream_t stream) {
   using C = Cfg<E, EV, RBF>;
   CUtensorMap tq, tk, tv;
   if (!make_map_rows(&tq, a.q, E, a.L, static_cast<long long>(a.N) * a.Hq, BM)) return -13;
@@ -848,6 +858,8 @@ int launch_impl(const AttnArgs& a, cudaStream_t stream) {
   pa.kv_start = a.kv_start;
   pa.kv_end = a.kv_end;
   pa.words = (a.S + 31) / 32;
+  pa.general = general;
+  pa.n_kt = (a.S + BN - 1) / BN;
   auto kern = prefill_kernel<E, EV, RBF, STREAM, EXT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return -13;
@@ -865,6 +877,32 @@ int launch_impl(const AttnArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+// A float [L, S] bias as keep bits for the EXT kernel: one warp per query row, one
+// 32-key word per iteration (lane l reads key 32w + l, the ballot of "entry == 0" is
+// the word).  general[i * n_kt + jb] records whether row i's key tile jb holds an
+// entry that is neither 0 nor -inf (+inf, NaN or a finite nonzero value); the kernel
+// adds the bias itself on those tiles, so the keep bits are exact wherever they are used.
+__global__ void __launch_bounds__(256) bias_bits_kernel(const float* __restrict__ bias, int L, int S, int words,
+                                                        int n_kt, uint32_t* __restrict__ bits,
+                                                        uint8_t* __restrict__ general) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= L) return;
+  const float* brow = bias + static_cast<size_t>(row) * S;
+  bool gen = false;
+  for (int w = 0; w < words; ++w) {
+    const int key = 32 * w + lane;
+    const float v = key < S ? __ldg(brow + key) : 0.f;
+    const uint32_t word = __ballot_sync(0xffffffffu, key < S && v == 0.f);
+    gen |= __any_sync(0xffffffffu, key < S && !(v == 0.f || v == -INFINITY));
+    if (lane == 0) bits[static_cast<size_t>(row) * words + w] = word;
+    if ((w & 3) == 3 || w == words - 1) {
+      if (lane == 0) general[static_cast<size_t>(row) * n_kt + (w >> 2)] = gen ? 1 : 0;
+      gen = false;
+    }
+  }
+}
 
 __global__ void exp2_poly_eval_kernel(const float* x, float* y, int n) {
   const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
@@ -884,15 +922,38 @@ int launch_exp2_poly_eval(const float* x, float* y, int n, cudaStream_t stream) 
 
 unsigned int take_status_prefill(cudaStream_t s) { return take_device_status_local(s); }
 
-int launch_prefill_bf16(const AttnArgs& a, cudaStream_t stream) {
+size_t prefill_workspace_bytes(const AttnArgs& a) {
+  // a float bias (outside the streaming mask's kernel) is converted to keep bits first
+  if (a.bias == nullptr || (a.mask_kind == MASK_STREAM && a.keep > 0)) return 0;
+  const size_t words = (static_cast<size_t>(a.S) + 31) / 32, n_kt = (static_cast<size_t>(a.S) + BN - 1) / BN;
+  return a.L * words * 4 + ((a.L * n_kt + 255) & ~static_cast<size_t>(255));
+}
+
+int launch_prefill_bf16(const AttnArgs& a0, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  AttnArgs a = a0;
   const bool r = a.rbf;
   const bool st = a.mask_kind == MASK_STREAM && a.keep > 0;
+  const uint8_t* general = nullptr;
+  if (a.bias != nullptr && !st) {
+    // the bias as keep bits plus per-tile "general" flags, then the EXT kernel
+    if (ws == nullptr || ws_bytes < prefill_workspace_bytes(a)) return -12;
+    const int words = (a.S + 31) / 32, n_kt = (a.S + BN - 1) / BN;
+    uint32_t* bits = static_cast<uint32_t*>(ws);
+    uint8_t* gen = reinterpret_cast<uint8_t*>(bits + static_cast<size_t>(a.L) * words);
+    bias_bits_kernel<<<(a.L + 7) / 8, 256, 0, stream>>>(a.bias, a.L, a.S, words, n_kt, bits, gen);
+    if (cudaGetLastError() != cudaSuccess) return -13;
+    a.mask_bits = bits;
+    general = gen;
+  }
   const bool ext = a.mask_bits != nullptr || a.kv_start != nullptr || a.kv_end != nullptr;
 #define ATTN_PREFILL_CASE(e, ev)                                                                              \
   if (a.E == e && a.Ev == ev) {                                                                               \
-    if (st) return r ? launch_impl<e, ev, true, true, false>(a, stream) : launch_impl<e, ev, false, true, false>(a, stream); \
-    if (ext) return r ? launch_impl<e, ev, true, false, true>(a, stream) : launch_impl<e, ev, false, false, true>(a, stream); \
-    return r ? launch_impl<e, ev, true, false, false>(a, stream) : launch_impl<e, ev, false, false, false>(a, stream); \
+    if (st) return r ? launch_impl<e, ev, true, true, false>(a, nullptr, stream)                              \
+                     : launch_impl<e, ev, false, true, false>(a, nullptr, stream);                            \
+    if (ext) return r ? launch_impl<e, ev, true, false, true>(a, general, stream)                             \
+                      : launch_impl<e, ev, false, false, true>(a, general, stream);                           \
+    return r ? launch_impl<e, ev, true, false, false>(a, nullptr, stream)                                     \
+             : launch_impl<e, ev, false, false, false>(a, nullptr, stream);                                   \
   }
   ATTN_PREFILL_CASE(64, 64)
   ATTN_PREFILL_CASE(128, 128)

@@ -43,6 +43,10 @@ METRIC = "attn fwd TFLOP/s (prefill), KV-read GB/s (decode), % of B200 roofline"
 DEFAULT_WORKLOAD = "dot_causal_2k_bf16"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# fp32 FMA-pipe roofline of the exact-fp32 path: measured FFMA throughput per SM per
+# clock on this B200 (a dependent-free FFMA stream, 4 warps per SM) x 2 flops x SMs x
+# the maximum SM clock
+FFMA_PER_CLK_SM = 122
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
 # dominant kernel from one ncu capture of the same kernel build; the capture
@@ -131,6 +135,10 @@ def work_units(r: sw.Recipe):
     if r.backward:
         # S^T, dP^T, dV, dK and dQ products: 2 (3E + 2Ev) flops per visible pair
         return 2 * (3 * r.E + 2 * r.Ev) * visible_pairs_total(r) * r.Hq, "TFLOP/s", "tensor"
+    if r.dtype == "f32":
+        # exact fp32 on the FMA pipe; a bias mask cannot skip work, so its pairs are counted
+        pairs = r.N * visible_pairs(r) if r.bias != "none" else visible_pairs_total(r)
+        return 2 * (r.E + r.Ev) * pairs * r.Hq, "TFLOP/s", "fma"
     flops = 2 * (r.E + r.Ev) * visible_pairs_total(r) * r.Hq
     return flops, "TFLOP/s", "tensor"
 
@@ -201,6 +209,17 @@ class ClockSampler:
         med = statistics.median(self.samples) if self.samples else None
         return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
                 "samples": len(self.samples)}
+
+
+def max_sm_mhz(device_index: int = 0) -> int:
+    """The GPU's maximum SM clock (NVML, read only); 1965 MHz, the B200's, if NVML is unavailable."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        return int(pynvml.nvmlDeviceGetMaxClockInfo(pynvml.nvmlDeviceGetHandleByIndex(device_index),
+                                                    pynvml.NVML_CLOCK_SM))
+    except Exception:  # noqa: BLE001
+        return 1965
 
 
 # ---------------------------------------------------------------------------
@@ -318,6 +337,11 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
     if bound == "tensor":
         peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         punit = "TFLOP/s"
+    elif bound == "fma":
+        props = torch.cuda.get_device_properties(torch.cuda.current_device())
+        max_mhz = (sampler.max_mhz if sampler and sampler.max_mhz else None) or max_sm_mhz()
+        peak = round(FFMA_PER_CLK_SM * 2 * props.multi_processor_count * max_mhz * 1e6 / 1e12, 2)
+        punit = "TFLOP/s"
     else:
         peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         punit = "GB/s"
@@ -327,8 +351,8 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
         "recipe": r, "amount": amount, "unit": unit, "secs_max": secs_max, "secs": secs,
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": punit,
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured"
-                     else "fallback"},
+                     "peak_source": ("derived: FFMA/clk/SM x 2 x SMs x max SM clock" if bound == "fma" else
+                                     f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback")},
         "launches_per_step": 2 if (is_decode(r) or r.backward) else 1,  # decode: partial + combine; backward: pre + main
         "clocks": sampler.summary() if sampler else None,
         "tensors": t, "out": out, "lse": lse, "dout": dout if r.backward else None,
@@ -535,7 +559,8 @@ def ours(args):
     extra = {}
     if not args.no_extra:
         import dataclasses
-        names = [n for n in sw.RECIPES if n != args.workload and sw.RECIPES[n].dtype == "bf16"]
+        # every reference workload but the tiny fp32 parity case
+        names = [n for n in sw.RECIPES if n != args.workload and n != "tiny_rbf_sink_causal_f32"]
         runs = []
         # steady-state control: the bench workload's kernel (dot, E=128) on one long
         # non-causal sequence, where per-item pipeline fill and drain are amortised

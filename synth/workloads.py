@@ -235,7 +235,7 @@ class Recipe:
     backward: bool = False    # the measured step is the backward pass (dout: N(0,1) draws of its own stream)
     sink: str = "none"    # "none", "fixed", "normal"
     sink_values: tuple = ()
-    bias: str = "none"    # "none" or "random10"
+    bias: str = "none"    # "none", "random10" or "mixed" (see bias_matrix)
     registers: int = 0    # zero K/V rows prepended (RBF workload)
     key_lognormal: bool = False
     sinusoid_pe: bool = False
@@ -334,15 +334,28 @@ def sink_logits(r: Recipe):
 
 
 def bias_matrix(r: Recipe):
-    """Additive [L, S] float32 bias or None.  random10: each entry is -inf with
-    probability 0.1 (uniform draw u < 0.1), 0 otherwise; the diagonal j == i is
-    always 0."""
+    """Additive [L, S] float32 bias or None.
+
+    random10: each entry is -inf with probability 0.1 (uniform draw u < 0.1), 0
+    otherwise; the diagonal j == i is always 0.
+    mixed: the random10 pattern, and on the 128 x 128 blocks with
+    (i // 128 + j // 128) odd every entry that is not -inf takes the finite value
+    4 u' - 2 in [-2, 2), u' the (L*S + i*S + j)-th draw of the same stream.  Half
+    the blocks thus hold general additive values and half only 0 / -inf.
+    """
     if r.bias == "none":
         return None
-    u = uniform_f64(stream_key(r.seed, STREAM_BIAS), 0, r.L * r.S).reshape(r.L, r.S)
+    key = stream_key(r.seed, STREAM_BIAS)
+    u = uniform_f64(key, 0, r.L * r.S).reshape(r.L, r.S)
     b = np.where(u < 0.1, -np.inf, 0.0)
     idx = np.arange(min(r.L, r.S))
     b[idx, idx] = 0.0
+    if r.bias == "mixed":
+        u2 = uniform_f64(key, r.L * r.S, r.L * r.S).reshape(r.L, r.S)
+        blk = ((np.arange(r.L)[:, None] // 128) + (np.arange(r.S)[None, :] // 128)) % 2 == 1
+        b = np.where(blk & np.isfinite(b), 4.0 * u2 - 2.0, b)
+    elif r.bias != "random10":
+        raise ValueError(f"unknown bias kind {r.bias!r}")
     return b.astype(np.float32)
 
 

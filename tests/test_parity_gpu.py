@@ -63,6 +63,13 @@ PREFILL_CASES = [
       window=128, keep=16, sink="normal", scale=0.0884),
     R("p_stream_w1_keep1_520", L=520, S=520, mask_kind="streaming", window=1, keep=1),
     R("p_stream_keep256_w128_1100", L=1100, S=1100, N=2, mask_kind="streaming", window=128, keep=256),
+    # a float bias is turned into keep bits before the kernel; blocks holding finite
+    # nonzero entries are flagged and add the bias values themselves
+    R("p_dot_bias_mixed_causal_300_e128_g2", L=300, S=300, E=128, Ev=128, Hq=4, H=2, mask_kind="causal",
+      bias="mixed", sink="normal", scale=0.0884),
+    R("p_rbf_bias_mixed_window_L260_S401", L=260, S=401, Hq=2, H=1, mode="rbf", mask_kind="window", window=200,
+      bias="mixed", scale=0.05),
+    R("p_dot_bias_mixed_none_L130_S257_sink", L=130, S=257, bias="mixed", sink="normal"),
 ]
 
 FP32_CASES = [

@@ -152,3 +152,21 @@ def test_keep_matrix_matches_random10_bias_and_padding_ranges():
     ks, ke = sw.kv_ranges(p)
     assert ks.min() >= 0 and ks.max() < 250 and ke.min() > 900 and ke.max() <= 1000 and len(set(ks)) > 10
     assert sw.kv_ranges(base) == (None, None)
+
+
+def test_mixed_bias_blocks():
+    """The mixed bias: -inf where random10 puts it, finite values in [-2, 2) on the odd
+    128 x 128 blocks, exact zeros elsewhere; the diagonal is never -inf."""
+    r = sw.Recipe("mixed", N=1, Hq=1, H=1, L=300, S=520, E=64, Ev=64, dtype="bf16", mode="dot", scale=0.125,
+                  mask_kind="none", bias="mixed", seed=9)
+    b = sw.bias_matrix(r)
+    import dataclasses
+    base = sw.bias_matrix(dataclasses.replace(r, name="r10", bias="random10"))
+    assert np.array_equal(np.isneginf(b), np.isneginf(base))
+    odd = ((np.arange(r.L)[:, None] // 128) + (np.arange(r.S)[None, :] // 128)) % 2 == 1
+    fin = np.isfinite(b)
+    assert np.all(b[fin & ~odd] == 0.0)
+    vals = b[fin & odd]
+    assert vals.size > 0 and vals.min() >= -2.0 and vals.max() < 2.0 and np.count_nonzero(vals) == vals.size
+    assert np.all(np.isfinite(np.diagonal(b)))
+    assert np.array_equal(b, sw.bias_matrix(r))

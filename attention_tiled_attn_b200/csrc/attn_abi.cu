@@ -321,7 +321,7 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
     case ATTN_ERR_DEVICE: return "device is not compute capability 10.x (B200)";
     case ATTN_ERR_SCRATCH_LIMIT: return "the call needs more scratch than the fixed no-allocation area holds";
-    case ATTN_ERR_NOT_DECODE: return "not a decode-shaped bf16 dot-score call ((Hq/H)*L must be <= 16)";
+    case ATTN_ERR_NOT_DECODE: return "not a decode-shaped bf16 call ((Hq/H)*L must be <= 16)";
     default: return "unknown status";
   }
 }

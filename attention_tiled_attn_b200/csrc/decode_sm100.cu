@@ -7,9 +7,17 @@
 // work list is split evenly across a persistent grid (one CTA per SM): CTA b
 // takes chunks [b*T/G, (b+1)*T/G), which may span the end of one unit and the
 // start of the next.  For each unit segment it writes a partial
-// (m, l, acc[Ev]) per query row; the combine kernel merges the partials of
-// each unit and adds the sink logit (page "Attention Sink" §4.2: the sink
-// joins the denominator only).
+// (m, l, acc[Ev]) per query row into slot b + u (CTA b, unit u: the pairs are
+// distinct and each unit's slots are consecutive) and counts it in a per-unit
+// arrival counter; the CTA whose count completes the unit merges all of the
+// unit's partials (one warp per query row) and adds the sink logit (page
+// "Attention Sink" §4.2: the sink joins the denominator only).  The counters are
+// zeroed before each launch; there is no second kernel.
+//
+// RBF variant: the score is -scale ||q - k||^2 in the expanded frame
+// 2 scale q.k - scale ||k||^2 (page "Dot-Product Attention을 거리 기반
+// RBF-Attention으로 교체한 실험기", 섹션별 상세); each consumer warp computes
+// ||k||^2 of its 16 keys from the staged K chunk.
 //
 // Per CTA: one TMA producer warp streams K and V chunks (3-D tensor maps,
 // 128-byte swizzle, zero fill past S) through a ring of stages; four consumer
@@ -66,7 +74,7 @@ struct DecodeParams {  // 128 bytes: kept at that size, the kernels' code genera
   int kb_win;       // first chunk after the head part (the window's; the first visible one otherwise)
   int nc;           // chunks per unit (head part + window part)
   int G;            // persistent CTAs
-  int max_segs;     // partial slots per CTA
+  int n_units;      // N * H
   float c_dot;      // scale * log2e
   int keep;         // streaming mask: initial keys every later query sees
   int nc_head;      // streaming mask: chunks of the kept initial keys (0 otherwise)
@@ -102,6 +110,8 @@ struct DCfg {
 };
 
 __device__ __forceinline__ long long seg_start(long long b, long long T, int G) { return (b * T) / G; }
+// The CTA whose chunk range [seg_start(b), seg_start(b + 1)) holds chunk c.
+__device__ __forceinline__ long long cta_of(long long c, long long T, int G) { return ((c + 1) * G - 1) / T; }
 
 // First key of a unit's local chunk.  STREAM (the streaming mask with kept keys,
 // a compile-time switch): the head part, then the window part.
@@ -148,16 +158,86 @@ __device__ __forceinline__ uint32_t sw_off(int row, int c16) {
   return (c16 >> 3) * (DC * 128) + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
 }
 
-template <int E, int EV, bool STREAM, bool GATHER, bool EXT>
+// The merge of one unit's partials for query row r, by one warp, 32 segments at a
+// time: lane j reads segment j's (m, l), shuffles reduce the block's maximum and
+// denominator, and each lane accumulates EV/32 output columns over the block's
+// segments with vector loads.  The sink joins the denominator only.  The partials
+// were written by other CTAs: they are read through L2 (ld.global.cg).
+template <int EV>
+__device__ __forceinline__ void combine_row(const DecodeParams& p, long long u, int r, int lane) {
+  constexpr int PER = EV / 32;  // output columns per lane
+  const int n = static_cast<int>(u / p.H), kvh = static_cast<int>(u % p.H);
+  const long long b0 = cta_of(u * p.nc, p.T, p.G), b1 = cta_of(u * p.nc + p.nc - 1, p.T, p.G);
+  const int nseg = static_cast<int>(b1 - b0 + 1);
+  const size_t slot0 = static_cast<size_t>(b0 + u);  // the unit's segments: slots slot0 .. slot0 + nseg - 1
+  const int hq = kvh * p.group + r / p.L;
+  const int i = r % p.L;
+  const float s2 = p.sink ? p.sink[hq] * LOG2E : -INFINITY;
+  float M = s2, l = 0.f;
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  for (int k0 = 0; k0 < nseg; k0 += 32) {
+    // lane j holds segment k0 + j's (m, l); the block's maximum rescales what came before
+    float2 ml = make_float2(-INFINITY, 0.f);
+    if (k0 + lane < nseg) ml = __ldcg(reinterpret_cast<const float2*>(p.ws_ml + ((slot0 + k0 + lane) * 16 + r) * 2));
+    float bm = ml.x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+    const float Mn = fmaxf(M, bm);
+    if (Mn == -INFINITY) continue;
+    if (Mn > M) {
+      const float sc = ex2(M - Mn);  // 0 while M is -inf
+      l *= sc;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) acc[e] *= sc;
+      M = Mn;
+    }
+    const float a = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
+    float la = a * ml.y;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) la += __shfl_xor_sync(0xffffffffu, la, o);
+    l += la;
+    const int cnt = min(32, nseg - k0);
+#pragma unroll 8
+    for (int j = 0; j < cnt; ++j) {
+      const float aj = __shfl_sync(0xffffffffu, a, j);
+      const float* src = p.ws_acc + ((slot0 + k0 + j) * 16 + r) * EV + lane * PER;
+      if constexpr (PER == 4) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+        acc[0] = fmaf(aj, v.x, acc[0]);
+        acc[1] = fmaf(aj, v.y, acc[1]);
+        acc[2] = fmaf(aj, v.z, acc[2]);
+        acc[3] = fmaf(aj, v.w, acc[3]);
+      } else {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
+        acc[0] = fmaf(aj, v.x, acc[0]);
+        acc[1] = fmaf(aj, v.y, acc[1]);
+      }
+    }
+  }
+  if (M != -INFINITY) l += ex2(s2 - M);
+  const float inv = (l > 0.f) ? 1.f / l : 0.f;
+  const size_t orow = (static_cast<size_t>(n) * p.Hq + hq) * p.L + i;
+  __nv_bfloat16* op = p.out + orow * EV + lane * PER;
+#pragma unroll
+  for (int e = 0; e < PER; e += 2)
+    *reinterpret_cast<uint32_t*>(op + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+  if (lane == 0 && p.lse) p.lse[orow] = (l > 0.f) ? (M + __log2f(l)) * LN2 : -INFINITY;
+}
+
+template <int E, int EV, bool STREAM, bool GATHER, bool EXT, bool RBF>
 __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
     decode_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const DecodeParams p, const ExtraArgs ga) {
   using C = DCfg<E, EV, GATHER>;
+  static_assert(!(GATHER && RBF), "listed-key decode takes the dot score");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t sb = (raw_addr + 1023u) & ~1023u;
   uint8_t* sp = smem_raw + (sb - raw_addr);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + C::OFF_MISC);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(sp + C::OFF_MISC + 4);  // fused combine
   auto full_bar = [&](int s) -> uint32_t { return sb + C::OFF_BAR + 8u * s; };
   auto empty_bar = [&](int s) -> uint32_t { return sb + C::OFF_BAR + 8u * (C::NSTAGE + s); };
 
@@ -295,7 +375,6 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
   float o[EV / 8][4];
   float m_run[2], l_run[2];
   long long cur_unit = -1;
-  int seg = 0;
   bool ok = true;
 
   auto load_q = [&](long long u) {
@@ -330,7 +409,7 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
   };
   float* merge_o = reinterpret_cast<float*>(sp + C::OFF_MERGE);
   float* merge_ml = reinterpret_cast<float*>(sp + C::OFF_ML);
-  auto flush = [&](long long u, int segi) {
+  auto flush = [&](long long u) {
     // per-warp state -> shared memory
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -349,7 +428,7 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
       }
     }
     consumer_bar();
-    const size_t slot = static_cast<size_t>(blockIdx.x) * p.max_segs + segi;
+    const size_t slot = static_cast<size_t>(blockIdx.x) + static_cast<size_t>(u);
     for (int x = threadIdx.x; x < p.R * EV; x += DWARPS * 32) {
       const int r = x / EV, e = x % EV;
       float M = -INFINITY;
@@ -370,13 +449,27 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
         p.ws_ml[(slot * 16 + r) * 2 + 1] = l;
       }
     }
+    // the CTA that finishes the unit's last segment merges all of its partials:
+    // publish this partial, count it, and let the count's last arrival combine
+    __threadfence();
+    consumer_bar();
+    if (threadIdx.x == 0) {
+      unsigned int* counters = reinterpret_cast<unsigned int*>(p.ws_ml + (static_cast<size_t>(p.G) + p.n_units) * 32);
+      const long long nseg = cta_of(u * p.nc + p.nc - 1, p.T, p.G) - cta_of(u * p.nc, p.T, p.G) + 1;
+      *last_flag = atomicAdd(counters + u, 1u) == static_cast<unsigned int>(nseg - 1) ? 1 : 0;
+    }
+    consumer_bar();
+    if (*last_flag) {
+      __threadfence();
+      for (int r = warp; r < p.R; r += DWARPS) combine_row<EV>(p, u, r, lane);
+    }
     consumer_bar();
   };
 
   for (long long c = c_begin; c < c_end; ++c) {
     const long long u = c / p.nc;
     if (u != cur_unit) {
-      if (cur_unit >= 0) flush(cur_unit, seg++);
+      if (cur_unit >= 0) flush(cur_unit);
       cur_unit = u;
       load_q(u);
       reset_state();
@@ -400,8 +493,11 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
     const int key0 = GATHER ? 0 : chunk_key0<STREAM>(p, static_cast<int>(c % p.nc)) + j0;
     const int* keys_c = reinterpret_cast<const int*>(sp + C::OFF_KEYS) + s * DC + j0;  // GATHER
 
-    // S = Q K^T for 16 keys (two n-tiles of 8)
+    // S = Q K^T for 16 keys (two n-tiles of 8).  RBF: the B fragments also give
+    // ||k||^2: lane l holds dimensions 2(l%4) + {0, 1, 8, 9} of each 16-wide slice
+    // for key l/4 of n-tile 0 (b0, b1) and of n-tile 1 (b2, b3)
     float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float kq0 = 0.f, kq1 = 0.f;  // partial squared norms of keys lane/4 and 8 + lane/4
     {
       const int mat = lane >> 3;
       const int krow = j0 + (mat >> 1) * 8 + (lane & 7);
@@ -411,16 +507,39 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
         ldsm_x4(kbuf + sw_off(krow, kk * 2 + (mat & 1)), b0, b1, b2, b3);
         mma16816(sc[0], qa[kk], b0, b1);
         mma16816(sc[1], qa[kk], b2, b3);
+        if constexpr (RBF) {
+          const uint32_t wv[4] = {b0, b1, b2, b3};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float lo = __uint_as_float(wv[q] << 16), hi = __uint_as_float(wv[q] & 0xFFFF0000u);
+            float& acc = q < 2 ? kq0 : kq1;
+            acc = fmaf(lo, lo, fmaf(hi, hi, acc));
+          }
+        }
       }
     }
-    // logits in base 2, masks and bias
+    // RBF: the four lanes of each key complete its norm; each lane then fetches the
+    // norms of the keys in its accumulator fragment (keys t*8 + cq + {0, 1})
+    float kn[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    if constexpr (RBF) {
+      kq0 += __shfl_xor_sync(0xffffffffu, kq0, 1);
+      kq0 += __shfl_xor_sync(0xffffffffu, kq0, 2);
+      kq1 += __shfl_xor_sync(0xffffffffu, kq1, 1);
+      kq1 += __shfl_xor_sync(0xffffffffu, kq1, 2);
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        kn[0][x] = __shfl_sync(0xffffffffu, kq0, 4 * (cq + x));
+        kn[1][x] = __shfl_sync(0xffffffffu, kq1, 4 * (cq + x));
+      }
+    }
+    // logits in base 2 (rbf: 2 scale q.k - scale ||k||^2), masks and bias
     const bool need_mask = GATHER || EXT || p.mask_kind != MASK_NONE || p.bias != nullptr || key0 + 16 > p.S;
 #pragma unroll
     for (int t = 0; t < 2; ++t)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int h = e >> 1;
-        float zz = sc[t][e] * p.c_dot;
+        float zz = RBF ? fmaf(sc[t][e], 2.f * p.c_dot, -kn[t][e & 1] * p.c_dot) : sc[t][e] * p.c_dot;
         if (need_mask) {
           const int key = GATHER ? keys_c[t * 8 + cq + (e & 1)] : key0 + t * 8 + cq + (e & 1);
           if constexpr (GATHER) {
@@ -489,62 +608,23 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
   }
   ok = __all_sync(0xffffffffu, ok);
   // all four consumer warps always reach this point together (same chunk list)
-  if (ok && cur_unit >= 0) flush(cur_unit, seg);
-}
-
-template <int EV>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
-  const int u = blockIdx.x;
-  const int n = u / p.H, kvh = u % p.H;
-  const long long c_first = static_cast<long long>(u) * p.nc;
-  const long long c_last = c_first + p.nc - 1;
-  auto cta_of = [&](long long c) -> long long {
-    long long b = (c * p.G) / p.T;
-    while (b + 1 < p.G && seg_start(b + 1, p.T, p.G) <= c) ++b;
-    while (b > 0 && seg_start(b, p.T, p.G) > c) --b;
-    return b;
-  };
-  const long long b0 = cta_of(c_first), b1 = cta_of(c_last);
-  for (int x = threadIdx.x; x < p.R * EV; x += blockDim.x) {
-    const int r = x / EV, e = x % EV;
-    const int hq = kvh * p.group + r / p.L;
-    const int i = r % p.L;
-    const float s2 = p.sink ? p.sink[hq] * LOG2E : -INFINITY;
-    float M = s2;
-    for (long long b = b0; b <= b1; ++b) {
-      const long long segi = u - seg_start(b, p.T, p.G) / p.nc;
-      const size_t slot = static_cast<size_t>(b) * p.max_segs + segi;
-      M = fmaxf(M, p.ws_ml[(slot * 16 + r) * 2]);
-    }
-    float acc = 0.f, l = 0.f;
-    if (M != -INFINITY) {
-      for (long long b = b0; b <= b1; ++b) {
-        const long long segi = u - seg_start(b, p.T, p.G) / p.nc;
-        const size_t slot = static_cast<size_t>(b) * p.max_segs + segi;
-        const float a = ex2(p.ws_ml[(slot * 16 + r) * 2] - M);
-        acc = fmaf(a, p.ws_acc[(slot * 16 + r) * EV + e], acc);
-        l = fmaf(a, p.ws_ml[(slot * 16 + r) * 2 + 1], l);
-      }
-      l += ex2(s2 - M);
-    }
-    const float inv = (l > 0.f) ? 1.f / l : 0.f;
-    const size_t orow = (static_cast<size_t>(n) * p.Hq + hq) * p.L + i;
-    p.out[orow * EV + e] = __float2bfloat16_rn(acc * inv);
-    if (e == 0 && p.lse) p.lse[orow] = (l > 0.f) ? (M + __log2f(l)) * LN2 : -INFINITY;
-  }
+  if (ok && cur_unit >= 0) flush(cur_unit);
 }
 
 struct DecodePlan {
-  int nc_head, kb_win, nc, G, max_segs;
+  int nc_head, kb_win, nc, G;
   long long T;
 };
+
+// Partial slots: one per (CTA, unit it touches), slot b + u.
+size_t partial_slots(const DecodePlan& d, const AttnArgs& a) {
+  return static_cast<size_t>(d.G) + static_cast<size_t>(a.N) * a.H;
+}
 
 // the even split of T chunks over a persistent grid, shared by both plans
 void split(DecodePlan& d, const AttnArgs& a, int num_sms) {
   d.T = static_cast<long long>(a.N) * a.H * d.nc;
   d.G = static_cast<int>(d.T < num_sms ? d.T : num_sms);
-  const long long per = (d.T + d.G - 1) / d.G;
-  d.max_segs = static_cast<int>((per + d.nc - 1) / d.nc + 1);
 }
 
 // GATHER: a unit's chunks are 64 consecutive entries of its key list
@@ -581,13 +661,13 @@ DecodePlan plan(const AttnArgs& a, int num_sms) {
   return d;
 }
 
-template <int E, int EV, bool STREAM, bool GATHER, bool EXT>
+template <int E, int EV, bool STREAM, bool GATHER, bool EXT, bool RBF>
 int launch_decode_impl(const AttnArgs& a, const ExtraArgs& ga, void* ws, size_t ws_bytes, int num_sms,
                        cudaStream_t stream) {
   using C = DCfg<E, EV, GATHER>;
   const DecodePlan d = GATHER ? plan_gather(a, ga.n_sel, num_sms) : plan(a, num_sms);
-  const size_t slots = static_cast<size_t>(d.G) * d.max_segs;
-  const size_t need = slots * 16 * (EV + 2) * sizeof(float);
+  const size_t slots = partial_slots(d, a);
+  const size_t need = slots * 16 * (EV + 2) * sizeof(float) + static_cast<size_t>(a.N) * a.H * sizeof(unsigned int);
   if (ws_bytes < need) return -12;
   CUtensorMap tk{}, tv{};  // GATHER reads K and V through plain pointers; its maps stay unused
   if (!GATHER) {
@@ -618,14 +698,16 @@ int launch_decode_impl(const AttnArgs& a, const ExtraArgs& ga, void* ws, size_t 
   p.nc = d.nc;
   p.T = d.T;
   p.G = d.G;
-  p.max_segs = d.max_segs;
+  p.n_units = a.N * a.H;
   p.c_dot = a.scale * LOG2E;
-  auto kern = decode_partial_kernel<E, EV, STREAM, GATHER, EXT>;
+  auto kern = decode_partial_kernel<E, EV, STREAM, GATHER, EXT, RBF>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return -13;
+  // per-unit arrival counters of the fused combine, after the partials
+  unsigned int* counters = reinterpret_cast<unsigned int*>(p.ws_ml + slots * 32);
+  if (cudaMemsetAsync(counters, 0, static_cast<size_t>(p.n_units) * sizeof(unsigned int), stream) != cudaSuccess)
+    return -13;
   kern<<<d.G, GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, C::SMEM_BYTES, stream>>>(tk, tv, p, ga);
-  if (cudaGetLastError() != cudaSuccess) return -13;
-  decode_combine_kernel<EV><<<a.N * a.H, 128, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? 0 : -13;
 }
 
@@ -633,16 +715,16 @@ int launch_decode_impl(const AttnArgs& a, const ExtraArgs& ga, void* ws, size_t 
 
 unsigned int take_status_decode(cudaStream_t s) { return take_device_status_local(s); }
 
-bool decode_eligible(const AttnArgs& a) { return (a.Hq / a.H) * a.L <= 16 && !a.rbf; }
+bool decode_eligible(const AttnArgs& a) { return (a.Hq / a.H) * a.L <= 16; }
 
 size_t decode_workspace_bytes(const AttnArgs& a, int num_sms) {
   const DecodePlan d = plan(a, num_sms);
-  return static_cast<size_t>(d.G) * d.max_segs * 16 * (a.Ev + 2) * sizeof(float);
+  return partial_slots(d, a) * 16 * (a.Ev + 2) * sizeof(float) + static_cast<size_t>(a.N) * a.H * sizeof(unsigned int);
 }
 
 size_t decode_gather_workspace_bytes(const AttnArgs& a, int n_sel, int num_sms) {
   const DecodePlan d = plan_gather(a, n_sel, num_sms);
-  return static_cast<size_t>(d.G) * d.max_segs * 16 * (a.Ev + 2) * sizeof(float);
+  return partial_slots(d, a) * 16 * (a.Ev + 2) * sizeof(float) + static_cast<size_t>(a.N) * a.H * sizeof(unsigned int);
 }
 
 int launch_decode_gather_bf16(const AttnArgs& a, const int* key_idx, int n_sel, void* ws, size_t ws_bytes,
@@ -653,7 +735,7 @@ int launch_decode_gather_bf16(const AttnArgs& a, const int* key_idx, int n_sel, 
   ga.v = static_cast<const __nv_bfloat16*>(a.v);
   ga.n_sel = n_sel;
 #define ATTN_GATHER_CASE(e, ev) \
-  if (a.E == e && a.Ev == ev) return launch_decode_impl<e, ev, false, true, false>(a, ga, ws, ws_bytes, num_sms, stream);
+  if (a.E == e && a.Ev == ev) return launch_decode_impl<e, ev, false, true, false, false>(a, ga, ws, ws_bytes, num_sms, stream);
   ATTN_GATHER_CASE(128, 128)
   ATTN_GATHER_CASE(64, 64)
   ATTN_GATHER_CASE(64, 128)
@@ -674,9 +756,14 @@ int launch_decode_bf16(const AttnArgs& a, void* ws, size_t ws_bytes, int num_sms
   xa.words = (a.S + 31) / 32;
 #define ATTN_DECODE_CASE(e, ev)                                                                              \
   if (a.E == e && a.Ev == ev) {                                                                              \
-    if (st) return launch_decode_impl<e, ev, true, false, false>(a, xa, ws, ws_bytes, num_sms, stream);    \
-    if (ext) return launch_decode_impl<e, ev, false, false, true>(a, xa, ws, ws_bytes, num_sms, stream);   \
-    return launch_decode_impl<e, ev, false, false, false>(a, xa, ws, ws_bytes, num_sms, stream);           \
+    if (a.rbf) {                                                                                             \
+      if (st) return launch_decode_impl<e, ev, true, false, false, true>(a, xa, ws, ws_bytes, num_sms, stream);  \
+      if (ext) return launch_decode_impl<e, ev, false, false, true, true>(a, xa, ws, ws_bytes, num_sms, stream); \
+      return launch_decode_impl<e, ev, false, false, false, true>(a, xa, ws, ws_bytes, num_sms, stream);         \
+    }                                                                                                        \
+    if (st) return launch_decode_impl<e, ev, true, false, false, false>(a, xa, ws, ws_bytes, num_sms, stream);   \
+    if (ext) return launch_decode_impl<e, ev, false, false, true, false>(a, xa, ws, ws_bytes, num_sms, stream);  \
+    return launch_decode_impl<e, ev, false, false, false, false>(a, xa, ws, ws_bytes, num_sms, stream);          \
   }
   ATTN_DECODE_CASE(128, 128)
   ATTN_DECODE_CASE(64, 64)

@@ -108,7 +108,7 @@ def visible_pairs_total(r: sw.Recipe) -> int:
 
 
 def is_decode(r: sw.Recipe) -> bool:
-    return r.dtype == "bf16" and r.mode == "dot" and (r.Hq // r.H) * r.L <= 16
+    return r.dtype == "bf16" and (r.Hq // r.H) * r.L <= 16
 
 
 def decode_keys(r: sw.Recipe) -> int:
@@ -590,6 +590,10 @@ def ours(args):
                              dataclasses.replace(r0, mask_kind="streaming", window=4096, keep=4)))
                 # exact attention over a 33x-sparse key selection (S/33 keys per KV head, random positions)
                 runs.append((name + ":top_k_33x", dataclasses.replace(r0, n_sel=r0.S // 33)))
+                # the RBF score on the same cache (key norms in the consumer warps), and one sequence
+                # (N=1: 8 KV heads, each split over ~18 CTAs, so the combine merges many partials)
+                runs.append((name + ":rbf", dataclasses.replace(r0, mode="rbf")))
+                runs.append((name + ":batch1", dataclasses.replace(r0, N=1)))
         for label, rr in runs:
             base = sw.RECIPES[rr.name]
             sw.RECIPES[rr.name] = rr
@@ -618,6 +622,9 @@ def ours(args):
                 extra[label + ":keep_bits_random10"]["time_vs_bias"] = round(
                     extra[label + ":keep_bits_random10"]["ms_per_step"] / extra[label + ":bias_random10"]["ms_per_step"],
                     4)
+            if label + ":rbf" in extra and extra[label]["mode"] == "dot":
+                extra[label + ":rbf"]["time_vs_dot"] = round(
+                    extra[label + ":rbf"]["ms_per_step"] / extra[label]["ms_per_step"], 4)
             if label + ":top_k_33x" in extra:
                 extra[label + ":top_k_33x"]["time_vs_dense"] = round(
                     extra[label + ":top_k_33x"]["ms_per_step"] / extra[label]["ms_per_step"], 4)

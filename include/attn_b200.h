@@ -66,7 +66,7 @@ typedef enum {
   ATTN_ERR_DEVICE_TIMEOUT = -14,/* a kernel gave up a bounded wait (see attn_device_status) */
   ATTN_ERR_DEVICE = -15,        /* the current device is not sm_100 */
   ATTN_ERR_SCRATCH_LIMIT = -16, /* attn_decode_fwd_noalloc: the call needs more scratch than the fixed area holds */
-  ATTN_ERR_NOT_DECODE = -17,    /* attn_decode_fwd_noalloc: not a decode-shaped bf16 call ((Hq/H)*L <= 16, dot) */
+  ATTN_ERR_NOT_DECODE = -17,    /* attn_decode_fwd_noalloc / attn_decode_indexed: not a decode-shaped bf16 call ((Hq/H)*L <= 16) */
   ATTN_ERR_KEEP = -18           /* keep_first < 0 (attn_fwd_streaming, attn_bwd), or kept keys without a window (attn_bwd) */
 } attn_status;
 
@@ -97,9 +97,13 @@ typedef enum {
  * synchronisation.  bf16 calls with (Hq/H)*L <= 16 run the split-key decode
  * path (partial kernel + combine kernel), which uses a library-owned device
  * workspace allocated stream-ordered on first need and grown monotonically;
- * all other bf16 calls run the single-kernel tcgen05 prefill path.
- * Calls on different streams may run concurrently except decode calls, which
- * share the workspace and must be ordered by the caller.
+ * all other bf16 calls run the tcgen05 prefill kernel.  With a float bias
+ * (outside the streaming mask) a pre-pass first turns the bias into packed
+ * keep bits plus per-128-key-tile flags for entries that are neither 0 nor
+ * -inf, in the same workspace; flagged tiles add the bias values, so every
+ * bias is applied exactly.  Calls on different streams may run concurrently
+ * except calls that use the workspace (decode calls and prefill calls with a
+ * bias), which must be ordered by the caller.
  */
 int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
              int N, int Hq, int H, int L, int S, int E, int Ev, float scale, int mode,
@@ -261,8 +265,8 @@ int attn_version(void);
 int attn_exp2_poly_eval(const float* x, float* y, int n, void* stream);
 
 /*
- * attn_decode_fwd_noalloc -- the decode path of attn_fwd (bf16, dot score,
- * (Hq/H)*L <= 16) without any device allocation.  The attention pages have
+ * attn_decode_fwd_noalloc -- the decode path of attn_fwd (bf16, dot or RBF
+ * score, (Hq/H)*L <= 16) without any device allocation.  The attention pages have
  * no counterpart to this entry point; it exists for callers that must not
  * allocate device memory while they run: services that reserve all GPU memory
  * at start-up and forbid later allocations (so latency stays predictable and

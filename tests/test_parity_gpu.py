@@ -104,6 +104,21 @@ DECODE_CASES = [
     R("d_stream_L2_S50_keep0_w10", L=2, S=50, mask_kind="streaming", window=10, keep=0),
     R("d_stream_many_units", L=1, S=3000, N=40, Hq=16, H=8, E=128, Ev=128, mask_kind="streaming", window=256,
       keep=4, scale=0.0884),
+    # the RBF score on the split-key path (key norms from the staged chunk)
+    R("d_rbf_L1_g4_S1000_sink", L=1, S=1000, E=128, Ev=128, N=2, Hq=8, H=2, mode="rbf", sink="normal",
+      scale=0.0884),
+    R("d_rbf_L4_g4_S777_causal_sink", L=4, S=777, Hq=8, H=2, mode="rbf", mask_kind="causal", sink="normal",
+      scale=0.05),
+    R("d_rbf_L2_S300_window_bias", L=2, S=300, Hq=2, H=1, mode="rbf", mask_kind="window", window=50,
+      bias="random10"),
+    R("d_rbf_lognormal_keys_L3_S400_e64_ev128", L=3, S=400, Hq=3, H=1, Ev=128, mode="rbf", mask_kind="causal",
+      key_lognormal=True, sink="normal"),
+    R("d_rbf_stream_L1_S5000_keep4_w1000_g4", L=1, S=5000, Hq=8, H=2, mode="rbf", mask_kind="streaming",
+      window=1000, keep=4, sink="normal", scale=0.05),
+    # one unit over every CTA: more than 32 partials per unit for the combine
+    R("d_rbf_one_unit_S19200_e128_ev64", L=1, S=19200, Hq=4, H=1, E=128, Ev=64, mode="rbf", sink="normal",
+      scale=0.05),
+    R("d_one_unit_L3_S20000_g5", L=3, S=20000, Hq=5, H=1, mask_kind="causal", sink="normal"),
 ]
 
 
@@ -124,6 +139,8 @@ PADDED_CASES = [
     R("d_pd_keep_L2_S777", L=2, S=777, Hq=4, H=2, keep_mask="random10", sink="normal"),
     R("d_pd_left_L1_S5000", L=1, S=5000, N=4, Hq=8, H=2, E=128, Ev=128, pad_left=0.5, scale=0.0884),
     R("d_pd_right_L4_g4_causal", L=4, S=900, N=3, Hq=8, H=2, mask_kind="causal", pad_right=0.6, keep_mask="random10"),
+    R("d_pd_rbf_keep_left_L2_S777", L=2, S=777, Hq=4, H=2, mode="rbf", keep_mask="random10", pad_left=0.3,
+      sink="normal", scale=0.05),
 ]
 
 
@@ -277,6 +294,9 @@ FULL_VARIANTS = [
     _variant("sink_gqa_window_16k_bf16", "streaming_keep4", mask_kind="streaming", keep=4),
     _variant("decode_sink_gqa_128k_bf16", "no_sink_control", sink="none"),
     _variant("decode_sink_gqa_128k_bf16", "streaming_keep4_w4096", mask_kind="streaming", window=4096, keep=4),
+    _variant("decode_sink_gqa_128k_bf16", "rbf", mode="rbf"),
+    _variant("decode_sink_gqa_128k_bf16", "batch1", N=1),
+    _variant("dot_causal_2k_bf16", "bias_mixed", bias="mixed"),
 ]
 
 

@@ -69,6 +69,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_exp2_poly_eval.restype = ci
     lib.attn_decode_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, ci, ci, vp, vp]
     lib.attn_decode_fwd_noalloc.restype = ci
+    lib.attn_test_wait_timeout.argtypes = [ci, vp]
+    lib.attn_test_wait_timeout.restype = ci
+    lib.attn_test_fail_workspace_allocs.argtypes = [ci]
+    lib.attn_test_fail_workspace_allocs.restype = ci
     lib.attn_decode_noalloc_scratch_bytes.argtypes = []
     lib.attn_decode_noalloc_scratch_bytes.restype = ctypes.c_size_t
     _lib = lib
@@ -359,6 +363,17 @@ def exp2_poly_eval(x: torch.Tensor) -> torch.Tensor:
 
 def decode_noalloc_scratch_bytes() -> int:
     return int(load_library().attn_decode_noalloc_scratch_bytes())
+
+
+def inject_wait_timeout(limit_cycles: int, stream: torch.cuda.Stream | None = None) -> int:
+    """Failure-path check: a kernel whose one bounded wait runs out (returns the launch status)."""
+    s = stream or torch.cuda.current_stream()
+    return load_library().attn_test_wait_timeout(int(limit_cycles), ctypes.c_void_p(s.cuda_stream))
+
+
+def inject_workspace_failures(count: int) -> int:
+    """Failure-path check: the next `count` workspace allocations fail (returns the status)."""
+    return load_library().attn_test_fail_workspace_allocs(int(count))
 
 
 def device_status(stream: torch.cuda.Stream | None = None) -> int:

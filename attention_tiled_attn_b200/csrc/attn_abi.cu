@@ -58,6 +58,7 @@ struct Workspace {
 
 std::mutex g_mutex;
 Workspace g_ws[MAX_DEVICES];
+int g_fail_allocs = 0;  // failure-path check: workspace allocations still to refuse (under g_mutex)
 int g_num_sms[MAX_DEVICES] = {0};
 int g_cc_major[MAX_DEVICES] = {0};
 
@@ -83,6 +84,10 @@ int ensure_workspace(int dev, size_t bytes, cudaStream_t stream, void** out) {
   std::lock_guard<std::mutex> lock(g_mutex);
   Workspace& w = g_ws[dev];
   if (w.bytes < bytes) {
+    if (g_fail_allocs > 0) {  // an injected allocation failure: the same return as a failed cudaMallocAsync
+      --g_fail_allocs;
+      return ATTN_ERR_WORKSPACE;
+    }
     if (w.ptr) cudaFreeAsync(w.ptr, stream);
     w.ptr = nullptr;
     w.bytes = 0;
@@ -353,6 +358,23 @@ int attn_device_status(void* stream_ptr) {
 }
 
 int attn_version(void) { return 10000; }
+
+int attn_test_wait_timeout(int limit_cycles, void* stream) {
+  using namespace attn;
+  if (limit_cycles < 1) return ATTN_ERR_BAD_SHAPE;
+  int dev = 0, sms = 0, major = 0;
+  if (device_info(&dev, &sms, &major) != ATTN_OK) return ATTN_ERR_CUDA;
+  if (major != 10) return ATTN_ERR_DEVICE;
+  return launch_wait_timeout_test(limit_cycles, static_cast<cudaStream_t>(stream));
+}
+
+int attn_test_fail_workspace_allocs(int count) {
+  using namespace attn;
+  if (count < 0) return ATTN_ERR_BAD_SHAPE;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_fail_allocs = count;
+  return ATTN_OK;
+}
 
 int attn_exp2_poly_eval(const float* x, float* y, int n, void* stream) {
   if (!x || !y) return ATTN_ERR_NULL_POINTER;

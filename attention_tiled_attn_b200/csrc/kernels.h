@@ -94,6 +94,8 @@ int launch_bwd_bf16(const BwdArgs& a, void* workspace, cudaStream_t stream);
 unsigned int take_status_bwd(cudaStream_t s);
 
 unsigned int take_status_prefill(cudaStream_t s);
+// A kernel whose one bounded wait runs out after limit_cycles (failure-path check).
+int launch_wait_timeout_test(int limit_cycles, cudaStream_t stream);
 unsigned int take_status_decode(cudaStream_t s);
 
 }  // namespace attn

@@ -920,6 +920,30 @@ int launch_exp2_poly_eval(const float* x, float* y, int n, cudaStream_t stream) 
   return cudaGetLastError() == cudaSuccess ? 0 : -13;
 }
 
+// Failure-path check: one thread waits on an mbarrier that nothing ever arrives
+// at, with a bounded wait of `limit` cycles, then records the timeout in this
+// file's status word exactly as the pipeline kernels' waits do, and returns.  No
+// copy or tensor-core work is in flight, so the early return is safe.
+__global__ void wait_timeout_test_kernel(long long limit) {
+  __shared__ __align__(8) unsigned long long bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  const long long t0 = clock64();
+  while (!mbar_try_wait(b, 0)) {
+    if (clock64() - t0 > limit) {
+      record_timeout();
+      return;
+    }
+  }
+}
+
+int launch_wait_timeout_test(int limit_cycles, cudaStream_t stream) {
+  wait_timeout_test_kernel<<<1, 32, 0, stream>>>(limit_cycles);
+  return cudaGetLastError() == cudaSuccess ? 0 : -13;
+}
+
 unsigned int take_status_prefill(cudaStream_t s) { return take_device_status_local(s); }
 
 size_t prefill_workspace_bytes(const AttnArgs& a) {

@@ -52,13 +52,9 @@ FFMA_PER_CLK_SM = 122
 # dominant kernel from one ncu capture of the same kernel build; the capture
 # command and counters are in profiles/.  Must be reset when the kernel changes.
 NCU_TRAFFIC_BYTES = {
-    "dot_causal_2k_bf16": 137_730_304 + 12_148_480,          # prefill_kernel<128,128,dot> (plain variant)
-    "sink_gqa_window_16k_bf16": 167_920_128 + 98_100_992,    # prefill_kernel<64,64,dot>
-    "rbf_registers_4k_bf16": 37_883_136 + 205_824,           # prefill_kernel<64,64,rbf>
-    # decode_partial_kernel<128,128>: batch-2 capture scaled by 16 to batch 32
-    "decode_sink_gqa_128k_bf16": 16 * (1_073_894_144 + 4_284_928),
-    # the same kernel's gather variant over 3971 listed keys (--select 3971), batch-2 capture scaled by 16
-    "decode_sink_gqa_128k_bf16:select3971": 16 * (32_867_072 + 5_376),
+    "dot_causal_2k_bf16": 132_508_416 + 11_135_232,          # prefill_kernel<128,128,dot> (plain variant)
+    # decode_partial_kernel<128,128> with the fused combine: batch-2 capture scaled by 16 to batch 32
+    "decode_sink_gqa_128k_bf16": 16 * (1_073_872_128 + 6_788_096),
     "dot_causal_2k_bf16:backward": 453_322_496 + 293_284_608,  # bwd_kernel<128,128> (--backward)
 }
 

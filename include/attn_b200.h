@@ -254,6 +254,32 @@ int attn_device_status(void* stream);
 int attn_version(void);
 
 /*
+ * Failure-path checks.  The attention pages have no counterpart to these two
+ * functions; they let a test drive the library's error paths without faulting
+ * or hanging a GPU.
+ *
+ * attn_test_wait_timeout -- launches on `stream` one thread that waits on a
+ * shared-memory barrier nothing ever arrives at, with a bounded wait of
+ * limit_cycles (>= 1) SM clock cycles.  The wait runs out, the thread records
+ * the timeout in the device status word as the pipeline kernels' bounded waits
+ * do, and the kernel returns; the next attn_device_status reports
+ * ATTN_ERR_DEVICE_TIMEOUT once and the context stays usable.  Returns
+ * ATTN_OK once launched, ATTN_ERR_BAD_SHAPE for limit_cycles < 1, or
+ * attn_fwd's device errors.
+ */
+int attn_test_wait_timeout(int limit_cycles, void* stream);
+
+/*
+ * attn_test_fail_workspace_allocs -- the next `count` (>= 0) allocations of the
+ * library workspace (the decode partials, a float bias's keep bits, the
+ * backward's per-row terms) fail as a failed cudaMallocAsync would: the call
+ * returns ATTN_ERR_WORKSPACE and launches nothing.  A workspace already large
+ * enough is not reallocated and does not fail.  0 clears the injection.
+ * Returns ATTN_OK, or ATTN_ERR_BAD_SHAPE for count < 0.
+ */
+int attn_test_fail_workspace_allocs(int count);
+
+/*
  * attn_exp2_poly_eval -- verification hook: y[i] = the prefill softmax's
  * software base-2 exponential of x[i] (device pointers, n floats).  A share of
  * the softmax exponentials is evaluated this way on the FMA pipe instead of

@@ -15,24 +15,31 @@
 //   dK_j += sum_i dS_ij q_i   (rbf: - k_j sum_i dS_ij)
 //   dsink_h = -sum_i 2^(s2_h - lse2_i) D_i (preprocess kernel)
 //
-// One CTA per (batch, KV head, 128-key tile) walks the query tiles of every
-// query head of its KV group that can see the tile, so dK and dV accumulate in
-// tensor memory and are stored once; dQ is accumulated in global memory with
-// vector reductions.  Per query tile five tcgen05 MMAs (M = N = 128):
-//   S^T  = K Q^T        (SS)      into TMEM columns [0, 128)
-//   dP^T = V dO^T       (SS)      into [128, 256)
-//   dV  += P^T dO       (TS: P^T as bf16 in [0, 64), dO MN-major)
-//   dK  += dS^T Q       (TS: dS^T as bf16 in [128, 192), Q MN-major)
-//   dQ   = dS K         (SS: dS written to shared memory by the compute warps in
-//                        the K-major layout the forward uses for Q; K MN-major)
-//                        into [0, E)
-// dV and dK live in [256, 256 + Ev) and [256 + Ev, 256 + Ev + E).  The dQ MMA
-// reuses the S^T columns; tcgen05 MMAs of one thread run in issue order, so it
-// follows the dV MMA that reads P^T there.
+// One CTA per (batch, KV head, 128-key tile) walks the 64-query tiles of every
+// query head of its KV group that can see the key tile, so dK and dV accumulate
+// in tensor memory and are stored once; dQ is accumulated in global memory with
+// reductions.  Per query tile b = it % 2 (two tiles in flight) five tcgen05 MMAs,
+// M = 128 keys (or head dimensions for dQ^T):
+//   S^T  = K Q^T      (SS, N = 64)             into TMEM columns S_b = [64 b, 64 b + 64)
+//   dP^T = V dO^T     (SS, N = 64)             into DP_b = [128 + 64 b, 192 + 64 b)
+//   dQ^T = K^T dS'^T  (SS, N = 64: K read MN-major, dS'^T MN-major)  into DP_b once dP^T is read
+//   dV  += P^T dO     (TS: P^T as bf16 pairs over the S_b columns, dO MN-major)
+//   dK  += dS'^T Q    (SS: dS'^T K-major, Q MN-major)
+// with dS' = dS / c_q; the factor c_q is applied where dQ and dK leave the kernel.
+// dS'^T (128 keys x 64 queries, bf16) is written to shared memory once per tile
+// (two buffers): read K-major it is the A operand of dK, read MN-major the B
+// operand of dQ^T.  dQ^T puts a head-dimension index on each TMEM lane, so one
+// reduction instruction of a warp covers 32 consecutive floats of a dQ row.  dV
+// and dK live in [256, 256 + Ev) and [256 + Ev, 256 + Ev + E).  tcgen05 MMAs of
+// one thread run in issue order, so S^T of tile it + 2 may be issued into the
+// columns the dV MMA of tile it still reads.
 //
-// Warps: 0-3 compute (thread = TMEM lane: a key row of S^T / dP^T, a query row
-// of dQ), 4 TMA producer, 5 MMA issuer.  Every wait is bounded.
+// Warps: 0-7 compute in two warpgroups (thread = TMEM lane = key row; warpgroup g
+// takes queries [32 g, 32 g + 32) of each tile), 8-11 read dQ^T out (thread =
+// head-dimension index), 12 TMA producer (Q, dO and the tile's lse2 and D), 13
+// MMA issuer.  Every wait is bounded.
 
+#include <climits>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -45,8 +52,12 @@ namespace attn {
 
 namespace {
 
-constexpr int TB = 128;  // keys per CTA tile and queries per query tile
-constexpr int BTHREADS = 6 * 32;
+constexpr int TB = 128;           // keys per CTA tile
+constexpr int QT = 64;            // queries per query tile
+constexpr int N_COMPUTE = 256;    // two warpgroups
+constexpr int W_DQ = N_COMPUTE / 32;  // first dQ readout warp
+constexpr int W_PRODUCER = W_DQ + 4, W_ISSUER = W_PRODUCER + 1;
+constexpr int BTHREADS = (W_ISSUER + 1) * 32;
 
 // tcgen05 instruction descriptor with the A major bit as well (bit 15: MN-major A)
 __host__ __device__ constexpr uint32_t idesc_ab(uint32_t M, uint32_t N, uint32_t a_mn, uint32_t b_mn) {
@@ -57,33 +68,38 @@ template <int E, int EV>
 struct BCfg {
   static constexpr int K_BYTES = TB * E * 2;
   static constexpr int V_BYTES = TB * EV * 2;
-  static constexpr int Q_BYTES = TB * E * 2;
-  static constexpr int DO_BYTES = TB * EV * 2;
-  static constexpr int NSTAGE = 2;
+  static constexpr int Q_BYTES = QT * E * 2;
+  static constexpr int DO_BYTES = QT * EV * 2;
+  static constexpr int LD_BYTES = 2 * QT * 4;                          // lse2 and D of the tile
+  static constexpr int NSTAGE = 4;
+  static constexpr int DS_BYTES = TB * QT * 2;                         // one dS'^T buffer
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + K_BYTES;
-  static constexpr int OFF_Q = OFF_V + V_BYTES;                       // [NSTAGE] Q tiles
-  static constexpr int OFF_DO = OFF_Q + NSTAGE * Q_BYTES;             // [NSTAGE] dO tiles
-  static constexpr int OFF_DS = OFF_DO + NSTAGE * DO_BYTES;           // dS, 128 queries x 128 keys, K-major
-  static constexpr int OFF_BAR = OFF_DS + TB * TB * 2;
-  static constexpr int NBAR = 1 + 2 * NSTAGE + 6;
+  static constexpr int OFF_Q = OFF_V + V_BYTES;                        // [NSTAGE] Q tiles
+  static constexpr int OFF_DO = OFF_Q + NSTAGE * Q_BYTES;              // [NSTAGE] dO tiles
+  static constexpr int OFF_DS = OFF_DO + NSTAGE * DO_BYTES;            // [2] dS'^T
+  static constexpr int OFF_LD = OFF_DS + 2 * DS_BYTES;                 // [NSTAGE] lse2[64], D[64]
+  static constexpr int OFF_BAR = OFF_LD + NSTAGE * LD_BYTES;
+  // barriers
+  static constexpr int B_KV = 0, B_QFULL = 1, B_QEMPTY = 1 + NSTAGE, B_SFULL = 1 + 2 * NSTAGE;
+  static constexpr int B_PFULL = B_SFULL + 2, B_DQFULL = B_SFULL + 4, B_DQEMPTY = B_SFULL + 6;
+  static constexpr int B_DKV = B_SFULL + 8, B_DRAIN = B_SFULL + 9;
+  static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  // barriers
-  static constexpr int B_KV = 0, B_QFULL = 1, B_QEMPTY = 1 + NSTAGE, B_SFULL = 1 + 2 * NSTAGE;
-  static constexpr int B_PFULL = B_SFULL + 1, B_DQFULL = B_SFULL + 2, B_DQEMPTY = B_SFULL + 3;
-  static constexpr int B_DKV = B_SFULL + 4, B_DRAIN = B_SFULL + 5;
+  static_assert(E >= 64 && E <= TB, "dQ^T takes the head dimension as M = 128");
+  static_assert(DS_BYTES >= 2 * TB * 4, "the rbf row-sum exchange reuses a dS'^T buffer");
   // TMEM columns
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + EV;
-  static constexpr uint32_t IDESC_S = idesc_ab(TB, TB, 0, 0);      // K Q^T and V dO^T
+  static constexpr uint32_t IDESC_S = idesc_ab(TB, QT, 0, 0);      // K Q^T and V dO^T
   static constexpr uint32_t IDESC_DV = idesc_ab(TB, EV, 0, 1);     // P^T dO
-  static constexpr uint32_t IDESC_DK = idesc_ab(TB, E, 0, 1);      // dS^T Q
-  static constexpr uint32_t IDESC_DQ = idesc_ab(TB, E, 0, 1);      // dS K
+  static constexpr uint32_t IDESC_DK = idesc_ab(TB, E, 0, 1);      // dS'^T Q
+  static constexpr uint32_t IDESC_DQ = idesc_ab(TB, QT, 1, 1);     // K^T dS'^T (rows >= E unused when E = 64)
 };
 
 struct BwdParams {
-  const float* lse2;   // [N*Hq*Lp] the forward's lse * log2e, -inf past L (Lp = L rounded up to 128)
+  const float* lse2;   // [N*Hq*Lp] the forward's lse * log2e; +inf past L and on rows that see no key
   const float* dsum;   // [N*Hq*Lp] D = dout . out, 0 past L
   float* dq;           // [N*Hq*L*E], accumulated (zeroed by the launcher)
   float* dk;           // [N*H*S*E]
@@ -108,16 +124,26 @@ __device__ __forceinline__ bool bwait(uint32_t bar, uint32_t parity, volatile in
   return false;
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
+__device__ __forceinline__ void red_add_f32(float* addr, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
 }
+
+// the two compute warpgroups only (named barrier 1)
+__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(N_COMPUTE) : "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// query tiles of head-local rows that can see some key of [k0, k0 + TB)
+// Plain (non-multicast) bulk copy of `bytes` (a multiple of 16, both addresses
+// 16-byte aligned) from global to this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// query tiles (of QT rows, head-local) that can see some key of [k0, k0 + TB)
 template <bool MX>
 __device__ __forceinline__ void query_tiles(const BwdParams& p, int k0, int& qt_lo, int& qt_hi) {
   const int off = p.S - p.L;
@@ -126,8 +152,53 @@ __device__ __forceinline__ void query_tiles(const BwdParams& p, int k0, int& qt_
   // i' - j < W, except that kept keys (streaming) stay visible to every later query
   if (p.mask_kind == MASK_WINDOW || (MX && p.mask_kind == MASK_STREAM && k0 >= p.keep))
     hi = min(p.L, k0 + TB - 1 + p.window - off);
-  qt_lo = lo / TB;
-  qt_hi = hi > lo ? (hi + TB - 1) / TB : qt_lo;
+  qt_lo = lo / QT;
+  qt_hi = hi > lo ? (hi + QT - 1) / QT : qt_lo;
+}
+
+// One warp's 32 x 32 block of a tile: this thread's key row j against the 32
+// queries qc .. qc + 31.  P = 2^(z2 - lse2) where visible, dS' = P (dP - D); P^T
+// goes back to TMEM as bf16 pairs, dS'^T to shared memory.  vis_lo / vis_w: the
+// visible query offsets of this row form [vis_lo, vis_lo + vis_w) (causal,
+// window and streaming masks, key range); MASKED adds that test (and the keep
+// bits) per element, RBF subtracts the key-norm term and sums dS' over the row.
+template <bool MX, bool MASKED, bool RBF>
+__device__ __forceinline__ void score_block(const BwdParams& p, const uint32_t (&sr)[32], const uint32_t (&dr)[32],
+                                            const float4* __restrict__ ls4, const float4* __restrict__ ds4,
+                                            int vis_lo, int vis_w, int qc, int j, float kn2, float& rowsum,
+                                            uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+  float pr[32], dsv[32];
+#pragma unroll
+  for (int e4 = 0; e4 < 8; ++e4) {
+    const float4 lv = ls4[e4], dv4 = ds4[e4];
+    const float l2[4] = {lv.x, lv.y, lv.z, lv.w}, dd[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = 4 * e4 + u;
+      const float nl = RBF ? -(l2[u] + kn2) : -l2[u];
+      float pe = ex2(fmaf(__uint_as_float(sr[e]), p.c_z, nl));
+      if constexpr (MASKED) {
+        bool vis = static_cast<unsigned>(e - vis_lo) < static_cast<unsigned>(vis_w);
+        if constexpr (MX) {
+          // keep bit (i, j): the 32 lanes of a warp hold 32 consecutive keys, one word (broadcast)
+          if (vis && p.bits != nullptr)
+            vis = (__ldg(p.bits + static_cast<size_t>(qc + e) * p.words + (j >> 5)) >> (j & 31)) & 1u;
+        }
+        pe = vis ? pe : 0.f;
+      }
+      pr[e] = pe;
+      dsv[e] = pe * (__uint_as_float(dr[e]) - dd[u]);
+    }
+  }
+  if constexpr (RBF) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) rowsum += dsv[e];
+  }
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    pk[e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
+    dk[e] = pack_bf16x2(dsv[2 * e], dsv[2 * e + 1]);
+  }
 }
 
 // MX: the streaming mask, keep bits or key padding is in use (a separate instantiation,
@@ -168,6 +239,9 @@ __global__ void __launch_bounds__(BTHREADS, 1)
   }
   const int n_qt = qt_hi - qt_lo;
   const int n_it = n_qt * p.group;  // (query head of the group, query tile) pairs
+  // tile it: query head kvh * group + it / n_qt, first query (qt_lo + it % n_qt) * QT
+  auto tile_q0 = [&](int it) { return (qt_lo + it % n_qt) * QT; };
+  auto tile_head = [&](int it) { return (static_cast<size_t>(n) * p.Hq + kvh * p.group + it / n_qt); };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -176,15 +250,17 @@ __global__ void __launch_bounds__(BTHREADS, 1)
       mbar_init(bar(C::B_QFULL + s), 1);
       mbar_init(bar(C::B_QEMPTY + s), 1);
     }
-    mbar_init(bar(C::B_SFULL), 1);
-    mbar_init(bar(C::B_PFULL), 128);
-    mbar_init(bar(C::B_DQFULL), 1);
-    mbar_init(bar(C::B_DQEMPTY), 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(C::B_SFULL + b), 1);
+      mbar_init(bar(C::B_PFULL + b), N_COMPUTE);
+      mbar_init(bar(C::B_DQFULL + b), 1);
+      mbar_init(bar(C::B_DQEMPTY + b), 128);
+    }
     mbar_init(bar(C::B_DKV), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == W_ISSUER) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -193,7 +269,7 @@ __global__ void __launch_bounds__(BTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == W_PRODUCER) {
     // ================= TMA producer =================
     if (lane == 0) {
       mbar_arrive_expect_tx(bar(C::B_KV), C::K_BYTES + C::V_BYTES);
@@ -204,15 +280,19 @@ __global__ void __launch_bounds__(BTHREADS, 1)
       for (int it = 0; it < n_it; ++it) {
         const int s = it % C::NSTAGE;
         if (!bwait(bar(C::B_QEMPTY + s), ((it / C::NSTAGE) & 1) ^ 1, abort_flag)) break;
-        const int hq = kvh * p.group + it / n_qt;
-        const int q0 = (qt_lo + it % n_qt) * TB;
-        const int qrow = n * p.Hq + hq;
-        mbar_arrive_expect_tx(bar(C::B_QFULL + s), C::Q_BYTES + C::DO_BYTES);
+        const int q0 = tile_q0(it);
+        const size_t head = tile_head(it);
+        const int qrow = static_cast<int>(head);
+        const uint32_t full = bar(C::B_QFULL + s);
+        mbar_arrive_expect_tx(full, C::Q_BYTES + C::DO_BYTES + C::LD_BYTES);
         for (int b = 0; b < E / 64; ++b)
-          tma_load_3d(sb + C::OFF_Q + s * C::Q_BYTES + b * (TB * 128), &tm_q, bar(C::B_QFULL + s), b * 64, q0, qrow);
+          tma_load_3d(sb + C::OFF_Q + s * C::Q_BYTES + b * (QT * 128), &tm_q, full, b * 64, q0, qrow);
         for (int b = 0; b < EV / 64; ++b)
-          tma_load_3d(sb + C::OFF_DO + s * C::DO_BYTES + b * (TB * 128), &tm_do, bar(C::B_QFULL + s), b * 64, q0,
-                      qrow);
+          tma_load_3d(sb + C::OFF_DO + s * C::DO_BYTES + b * (QT * 128), &tm_do, full, b * 64, q0, qrow);
+        // lse2 and D of the tile (padded rows: 256-byte aligned, inside the Lp-row head)
+        const size_t pad = head * p.Lp + q0;
+        bulk_load(sb + C::OFF_LD + s * C::LD_BYTES, p.lse2 + pad, QT * 4, full);
+        bulk_load(sb + C::OFF_LD + s * C::LD_BYTES + QT * 4, p.dsum + pad, QT * 4, full);
         issued = it + 1;
       }
       // drain: every issued copy has landed before exit
@@ -220,7 +300,7 @@ __global__ void __launch_bounds__(BTHREADS, 1)
       for (int it = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); it < issued; ++it)
         mbar_wait(bar(C::B_QFULL + it % C::NSTAGE), (it / C::NSTAGE) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == W_ISSUER) {
     // ================= tcgen05 issuer =================
     if (lane == 0) {
       bool ok = bwait(bar(C::B_KV), 0, abort_flag);
@@ -229,57 +309,134 @@ __global__ void __launch_bounds__(BTHREADS, 1)
       const uint32_t k_lo_kmaj = desc_lo(sb + C::OFF_K, 16);
       const uint32_t v_lo_kmaj = desc_lo(sb + C::OFF_V, 16);
       const uint32_t k_lo_mn = desc_lo(sb + C::OFF_K, TB * 128);
-      const uint32_t ds_lo_kmaj = desc_lo(sb + C::OFF_DS, 16);
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it % C::NSTAGE;
-        if (!bwait(bar(C::B_QFULL + s), (it / C::NSTAGE) & 1, abort_flag)) break;
-        if (it > 0 && !bwait(bar(C::B_DQEMPTY), (it - 1) & 1, abort_flag)) break;  // dQ of it-1 read
-        tc_fence_after();
-        const uint32_t q_lo_kmaj = desc_lo(sb + C::OFF_Q + s * C::Q_BYTES, 16);
-        const uint32_t do_lo_kmaj = desc_lo(sb + C::OFF_DO + s * C::DO_BYTES, 16);
-        // S^T = K Q^T, dP^T = V dO^T (K-major operands; K steps of 16 inside 64-column boxes)
+      // K-major operands step 16 along K inside 64-column boxes (of 128 key rows or 64 query rows)
+      auto koff = [](int kk, int box_bytes) -> uint32_t {
+        return static_cast<uint32_t>(((kk / 4) * box_bytes + (kk % 4) * 32) >> 4);
+      };
+      // S^T and dP^T of tile it into S_b / DP_b
+      auto issue_s = [&](int it) {
+        const uint32_t q_lo = desc_lo(sb + C::OFF_Q + (it % C::NSTAGE) * C::Q_BYTES, 16);
+        const uint32_t d = tmem + C::T_S + 64 * (it & 1);
 #pragma unroll
-        for (int kk = 0; kk < E / 16; ++kk) {
-          const uint32_t koff = ((kk / 4) * (TB * 128) + (kk % 4) * 32) >> 4;
-          mma_ss_h(tmem + C::T_S, k_lo_kmaj + koff, hi, q_lo_kmaj + koff, hi, C::IDESC_S, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < E / 16; ++kk)
+          mma_ss_h(d, k_lo_kmaj + koff(kk, TB * 128), hi, q_lo + koff(kk, QT * 128), hi, C::IDESC_S, kk > 0 ? 1u : 0u);
+      };
+      auto issue_dp = [&](int it) {
+        const uint32_t do_lo = desc_lo(sb + C::OFF_DO + (it % C::NSTAGE) * C::DO_BYTES, 16);
+        const uint32_t d = tmem + C::T_DP + 64 * (it & 1);
 #pragma unroll
-        for (int kk = 0; kk < EV / 16; ++kk) {
-          const uint32_t koff = ((kk / 4) * (TB * 128) + (kk % 4) * 32) >> 4;
-          mma_ss_h(tmem + C::T_DP, v_lo_kmaj + koff, hi, do_lo_kmaj + koff, hi, C::IDESC_S, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(C::B_SFULL));
-        if (!bwait(bar(C::B_PFULL), it & 1, abort_flag)) break;
-        tc_fence_after();
-        // dV += P^T dO, dK += dS^T Q (A from TMEM: 8 columns per 16 queries; B MN-major: 16 rows per step)
-        const uint32_t do_lo_mn = desc_lo(sb + C::OFF_DO + s * C::DO_BYTES, TB * 128);
-        const uint32_t q_lo_mn = desc_lo(sb + C::OFF_Q + s * C::Q_BYTES, TB * 128);
-#pragma unroll
-        for (int kk = 0; kk < TB / 16; ++kk)
-          mma_ts_h(tmem + C::T_DV, tmem + C::T_S + kk * 8, do_lo_mn + kk * 128, hi, C::IDESC_DV,
-                   (it > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < EV / 16; ++kk)
+          mma_ss_h(d, v_lo_kmaj + koff(kk, TB * 128), hi, do_lo + koff(kk, QT * 128), hi, C::IDESC_S,
+                   kk > 0 ? 1u : 0u);
+      };
+      // the rest of tile it once its scores are consumed: dQ^T into DP_b, dV, dK
+      auto issue_grads = [&](int it) {
+        const int b = it & 1, s = it % C::NSTAGE;
+        const uint32_t ds_base = sb + C::OFF_DS + b * C::DS_BYTES;
+        const uint32_t ds_lo_mn = desc_lo(ds_base, C::DS_BYTES);  // one 64-query box: the MN stride is unused
+        const uint32_t ds_lo_kmaj = desc_lo(ds_base, 16);
 #pragma unroll
         for (int kk = 0; kk < TB / 16; ++kk)
-          mma_ts_h(tmem + C::T_DK, tmem + C::T_DP + kk * 8, q_lo_mn + kk * 128, hi, C::IDESC_DK,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-        // dQ = dS K: A = dS in shared memory (K-major over keys), B = K read MN-major (16 keys per step)
+          mma_ss_h(tmem + C::T_DP + 64 * b, k_lo_mn + kk * 128, hi, ds_lo_mn + kk * 128, hi, C::IDESC_DQ,
+                   kk > 0 ? 1u : 0u);
+        mma_commit(bar(C::B_DQFULL + b));
+        // dV += P^T dO: query q's bf16 pair sits in column 64 b + 32 (q / 32) + (q % 32) / 2
+        const uint32_t do_lo_mn = desc_lo(sb + C::OFF_DO + s * C::DO_BYTES, QT * 128);
+        const uint32_t q_lo_mn = desc_lo(sb + C::OFF_Q + s * C::Q_BYTES, QT * 128);
 #pragma unroll
-        for (int kk = 0; kk < TB / 16; ++kk) {
-          const uint32_t koff = ((kk / 4) * (TB * 128) + (kk % 4) * 32) >> 4;
-          mma_ss_h(tmem + C::T_S, ds_lo_kmaj + koff, hi, k_lo_mn + kk * 128, hi, C::IDESC_DQ, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < QT / 16; ++kk)
+          mma_ts_h(tmem + C::T_DV, tmem + C::T_S + 64 * b + 32 * (kk / 2) + 8 * (kk % 2), do_lo_mn + kk * 128, hi,
+                   C::IDESC_DV, (it > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS'^T Q (A K-major over the tile's 64 queries: 32 bytes per step)
+#pragma unroll
+        for (int kk = 0; kk < QT / 16; ++kk)
+          mma_ss_h(tmem + C::T_DK, ds_lo_kmaj + kk * 2, hi, q_lo_mn + kk * 128, hi, C::IDESC_DK,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar(C::B_QEMPTY + s));  // Q, dO, lse2 and D of this stage are no longer read
+      };
+      // tiles 0 and 1 start at once (their buffers are fresh)
+      for (int it = 0; ok && it < 2 && it < n_it; ++it) {
+        ok = bwait(bar(C::B_QFULL + it % C::NSTAGE), (it / C::NSTAGE) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(it);
+        issue_dp(it);
+        mma_commit(bar(C::B_SFULL + (it & 1)));
+      }
+      // Two event streams, served as they come: PFULL(np) (tile np's scores consumed) and
+      // DQEMPTY of tile ndp - 2 (DP_b free again for dP^T of tile ndp).
+      int np = 0, ndp = 2;
+      long long t_last = clock64();
+      while (ok && np < n_it) {
+        bool progress = false;
+        if (ndp < n_it && ndp - 2 < np && mbar_test(bar(C::B_DQEMPTY + (ndp & 1)), ((ndp - 2) >> 1) & 1)) {
+          tc_fence_after();
+          issue_dp(ndp);  // S^T of tile ndp went out with the gradients of tile ndp - 2
+          mma_commit(bar(C::B_SFULL + (ndp & 1)));
+          ++ndp;
+          progress = true;
         }
-        mma_commit(bar(C::B_DQFULL));
-        mma_commit(bar(C::B_QEMPTY + s));  // Q and dO of this stage are no longer read
+        if (mbar_test(bar(C::B_PFULL + (np & 1)), (np >> 1) & 1)) {
+          tc_fence_after();
+          issue_grads(np);
+          if (np + 2 < n_it) {
+            if (!bwait(bar(C::B_QFULL + (np + 2) % C::NSTAGE), ((np + 2) / C::NSTAGE) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(np + 2);  // after the dV MMA that reads P^T in these columns
+          }
+          ++np;
+          progress = true;
+        }
+        if (progress) {
+          t_last = clock64();
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (clock64() - t_last > WAIT_LIMIT_CYCLES) {
+          record_timeout();
+          *abort_flag = 1;
+          ok = false;
+        }
       }
       mma_commit(bar(C::B_DKV));
       mma_commit(bar(C::B_DRAIN));
       mbar_wait(bar(C::B_DRAIN), 0);
     }
+  } else if (warp >= W_DQ) {
+    // ================= dQ^T readout: lane = head-dimension index, column = query =================
+    const int t = threadIdx.x & 127;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const bool has_rows = (warp & 3) * 32 < E;  // lanes >= E hold nothing (E = 64)
+    for (int it = 0; it < n_it; ++it) {
+      const int b = it & 1;
+      if (!__all_sync(0xffffffffu, bwait(bar(C::B_DQFULL + b), (it >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      if (has_rows) {
+        const int q0 = tile_q0(it);
+        float* dq_col = p.dq + (tile_head(it) * p.L + q0) * E + t;
+        const int lim = p.L - q0;
+#pragma unroll 1
+        for (int ch = 0; ch < QT / 32; ++ch) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + C::T_DP + 64 * b + 32 * ch, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (32 * ch + e < lim)
+              red_add_f32(dq_col + static_cast<size_t>(32 * ch + e) * E, p.c_q * __uint_as_float(r[e]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DQEMPTY + b));
+    }
   } else {
-    // ================= compute warps 0-3 =================
-    const int t = threadIdx.x;  // TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int j = k0 + t;       // this thread's key row of S^T / dP^T
+    // ================= compute warpgroups =================
+    const int t = threadIdx.x & (TB - 1);  // TMEM lane
+    const int g = threadIdx.x >> 7;        // warpgroup: queries [32 g, 32 g + 32) of each tile
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int j = k0 + t;                  // this thread's key row of S^T / dP^T
     const int off = p.S - p.L;
     // rbf: the key-norm term of this key, in base-2 logit units
     float kn2 = 0.f;
@@ -303,174 +460,146 @@ __global__ void __launch_bounds__(BTHREADS, 1)
       }
       kn2 = acc * p.c_kn;
     }
-    float ds_rowsum = 0.f;  // rbf: sum_i dS_ij of this key
+    // keys outside [0, S) (and, with padding, outside [ks, ke)) see no query
+    const bool key_ok = j < p.S && (!MX || (j >= ks && j < ke));
+    float ds_rowsum = 0.f;  // rbf: sum_i dS'_ij of this key over this warpgroup's queries
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      const int hq = kvh * p.group + it / n_qt;
-      const int q0 = (qt_lo + it % n_qt) * TB;
-      const size_t rowbase = (static_cast<size_t>(n) * p.Hq + hq) * p.L;
-      const size_t padbase = (static_cast<size_t>(n) * p.Hq + hq) * p.Lp + q0;  // 16-byte aligned
-      if (!__all_sync(0xffffffffu, bwait(bar(C::B_SFULL), it & 1, abort_flag))) {
+      const int b = it & 1, s = it % C::NSTAGE;
+      const int qc = tile_q0(it) + 32 * g;  // this warpgroup's first query
+      // SFULL: S^T and dP^T in TMEM; QFULL (already complete): lse2 and D of the stage are visible here
+      if (!__all_sync(0xffffffffu, bwait(bar(C::B_SFULL + b), (it >> 1) & 1, abort_flag) &&
+                                       bwait(bar(C::B_QFULL + s), (it / C::NSTAGE) & 1, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const bool key_ok = j < p.S;
-      // dS element (query c, this key t) of the K-major tile: box t/64, row c, 16-byte unit (t%64)/8 swizzled by c
-      uint8_t* ds_col = sp + C::OFF_DS + (t >> 6) * (TB * 128) + (t & 7) * 2;
-      const int ds_unit = (t & 63) >> 3;
-#pragma unroll 1
-      for (int ch = 0; ch < TB / 32; ++ch) {
-        // the chunk's lse2 and D (every thread reads the same 256 bytes: L1 broadcast), issued first
-        float4 l4[8], d4[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          l4[u] = __ldg(reinterpret_cast<const float4*>(p.lse2 + padbase + ch * 32) + u);
-          d4[u] = __ldg(reinterpret_cast<const float4*>(p.dsum + padbase + ch * 32) + u);
-        }
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tmem + lane_base + C::T_S + ch * 32, sr);
-        tmem_ld32(tmem + lane_base + C::T_DP + ch * 32, dr);
-        tmem_wait_ld();
-        uint32_t pk[16], dk[16];
-        float dsv[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = ch * 32 + e;
-          const int i = q0 + c;
-          const float4 lv = l4[e >> 2], dv4 = d4[e >> 2];
-          const float l2 = (e & 3) == 0 ? lv.x : (e & 3) == 1 ? lv.y : (e & 3) == 2 ? lv.z : lv.w;
-          const float dd = (e & 3) == 0 ? dv4.x : (e & 3) == 1 ? dv4.y : (e & 3) == 2 ? dv4.z : dv4.w;
-          bool vis = key_ok && l2 != -INFINITY;  // -inf past L and on rows that see no key
-          if (p.mask_kind != MASK_NONE) vis = vis && j <= i + off;
-          if (p.mask_kind == MASK_WINDOW) vis = vis && (i + off - j) < p.window;
-          if constexpr (MX) {
-            if (p.mask_kind == MASK_STREAM) vis = vis && (j < p.keep || (i + off - j) < p.window);
-            vis = vis && j >= ks && j < ke;
-            // keep bit (i, j): the 32 lanes of a warp hold 32 consecutive keys, one word (broadcast)
-            if (vis && p.bits != nullptr)
-              vis = (__ldg(p.bits + static_cast<size_t>(i) * p.words + (j >> 5)) >> (j & 31)) & 1u;
-          }
-          const float z2 = fmaf(__uint_as_float(sr[e]), p.c_z, -kn2);
-          const float pr = vis ? ex2(z2 - l2) : 0.f;
-          const float ds = p.c_q * pr * (__uint_as_float(dr[e]) - dd);
-          dsv[e] = ds;
-          ds_rowsum += ds;
-          sr[e] = __float_as_uint(pr);
-        }
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          pk[e] = pack_bf16x2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
-          dk[e] = pack_bf16x2(dsv[2 * e], dsv[2 * e + 1]);
-        }
-        // P^T and dS^T as bf16 pairs: chunk ch goes to columns already read
-        tmem_st16(tmem + lane_base + C::T_S + ch * 16, pk);
-        tmem_st16(tmem + lane_base + C::T_DP + ch * 16, dk);
-        // dS into the K-major shared tile: one bf16 per query row (a warp's 32 keys fill 64 contiguous bytes)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = ch * 32 + e;
-          *reinterpret_cast<__nv_bfloat16*>(ds_col + c * 128 + ((ds_unit ^ (c & 7)) << 4)) = __float2bfloat16_rn(dsv[e]);
-        }
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tmem + lane_base + C::T_S + 64 * b + 32 * g, sr);
+      tmem_ld32(tmem + lane_base + C::T_DP + 64 * b + 32 * g, dr);
+      // visible queries of this key row: [lo, hi) as offsets from qc
+      const int jr = j - off - qc;  // causal: i >= j - off
+      int lo = p.mask_kind != MASK_NONE ? jr : INT_MIN / 2;
+      int hi = INT_MAX / 2;
+      if (p.mask_kind == MASK_WINDOW) hi = jr + p.window;
+      if constexpr (MX) {
+        if (p.mask_kind == MASK_STREAM && j >= p.keep) hi = jr + p.window;
       }
+      if (!key_ok) lo = 32;
+      const int lo_c = min(max(lo, 0), 32), hi_c = min(max(hi, 0), 32);
+      const int vis_w = max(hi_c - lo_c, 0);
+      const bool all_vis = __all_sync(0xffffffffu, vis_w == 32) && !(MX && p.bits != nullptr);
+      const float4* ls4 = reinterpret_cast<const float4*>(sp + C::OFF_LD + s * C::LD_BYTES) + 8 * g;
+      const float4* ds4 = ls4 + QT / 4;
+      uint32_t pk[16], dk[16];
+      tmem_wait_ld();
+      if (all_vis) {
+        if (p.rbf)
+          score_block<MX, false, true>(p, sr, dr, ls4, ds4, 0, 32, qc, j, kn2, ds_rowsum, pk, dk);
+        else
+          score_block<MX, false, false>(p, sr, dr, ls4, ds4, 0, 32, qc, j, kn2, ds_rowsum, pk, dk);
+      } else {
+        if (p.rbf)
+          score_block<MX, true, true>(p, sr, dr, ls4, ds4, lo_c, vis_w, qc, j, kn2, ds_rowsum, pk, dk);
+        else
+          score_block<MX, true, false>(p, sr, dr, ls4, ds4, lo_c, vis_w, qc, j, kn2, ds_rowsum, pk, dk);
+      }
+      // P^T as bf16 pairs over S^T columns this warpgroup has already read
+      tmem_st16(tmem + lane_base + C::T_S + 64 * b + 32 * g, pk);
+      // dS'^T row t of buffer b: this warpgroup's queries are 16-byte units 4 g .. 4 g + 3
+      uint8_t* ds_row = sp + C::OFF_DS + b * C::DS_BYTES + t * 128;
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        *reinterpret_cast<uint4*>(ds_row + (((4 * g + v) ^ (t & 7)) << 4)) =
+            make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
       tmem_wait_st();
-      fence_proxy_async_smem();  // the dS^T tile is read by the tensor core (async proxy)
+      fence_proxy_async_smem();  // dS'^T is read by the tensor core (async proxy)
       tc_fence_before();
-      mbar_arrive(bar(C::B_PFULL));
-      // dQ rows of this query tile: lane t = query q0 + t
-      if (!__all_sync(0xffffffffu, bwait(bar(C::B_DQFULL), it & 1, abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      {
-        const int i = q0 + t;
-        float* dq_row = p.dq + (rowbase + i) * E;
-#pragma unroll 1
-        for (int c = 0; c < E; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + C::T_S + c, r);
-          tmem_wait_ld();
-          if (i < p.L) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              red_add_v4(dq_row + c + e, __uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
-                         __uint_as_float(r[e + 3]));
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(bar(C::B_DQEMPTY));
+      mbar_arrive(bar(C::B_PFULL + b));
     }
-    // dK and dV of this key row
+    // dV (warpgroup 0) and dK (warpgroup 1) of this key row
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && n_it > 0 && __all_sync(0xffffffffu, bwait(bar(C::B_DKV), 0, abort_flag))) {
+    const bool grads_ready = ok && n_it > 0 && __all_sync(0xffffffffu, bwait(bar(C::B_DKV), 0, abort_flag));
+    // the two warpgroups' halves of sum_i dS'_ij (rbf), exchanged through a dS'^T buffer
+    // that no MMA reads any more once DKV has completed
+    float* red_s = reinterpret_cast<float*>(sp + C::OFF_DS);
+    if (grads_ready) red_s[g * TB + t] = ds_rowsum;
+    compute_bar();
+    if (grads_ready) ds_rowsum = red_s[t] + red_s[TB + t];
+    float* dv_row = p.dv + (static_cast<size_t>(nh) * p.S + j) * EV;
+    float* dk_row = p.dk + (static_cast<size_t>(nh) * p.S + j) * E;
+    if (grads_ready) {
       tc_fence_after();
       // tcgen05.ld is warp-collective: every lane loads, only rows j < S are stored
       const bool row_ok = j < p.S;
-      float* dv_row = p.dv + (static_cast<size_t>(nh) * p.S + j) * EV;
-      float* dk_row = p.dk + (static_cast<size_t>(nh) * p.S + j) * E;
+      if (g == 0) {
 #pragma unroll 1
-      for (int c = 0; c < EV; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + C::T_DV + c, r);
-        tmem_wait_ld();
-        if (row_ok) {
+        for (int c = 0; c < EV; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + C::T_DV + c, r);
+          tmem_wait_ld();
+          if (row_ok) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dv_row + c + e) = make_float4(
-                __uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-        }
-      }
-      const uint8_t* kt_s = sp + C::OFF_K;
-#pragma unroll 1
-      for (int c = 0; c < E; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + C::T_DK + c, r);
-        tmem_wait_ld();
-        float g[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) g[e] = __uint_as_float(r[e]);
-        if (p.rbf) {
-          // - k_j * sum_i dS_ij (k from the swizzled K tile: column c + e is 16-byte unit ((c+e)%64)/8 of box (c+e)/64)
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int col = c + 8 * u;
-            const uint4 w = *reinterpret_cast<const uint4*>(kt_s + (col / 64) * (TB * 128) + t * 128 +
-                                                            ((((col % 64) / 8) ^ (t & 7)) << 4));
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              g[8 * u + 2 * e] -= __uint_as_float(ws[e] << 16) * ds_rowsum;
-              g[8 * u + 2 * e + 1] -= __uint_as_float(ws[e] & 0xFFFF0000u) * ds_rowsum;
-            }
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dv_row + c + e) =
+                  make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                              __uint_as_float(r[e + 3]));
           }
         }
-        if (row_ok) {
+      } else {
+        const uint8_t* kt_s = sp + C::OFF_K;
+#pragma unroll 1
+        for (int c = 0; c < E; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + C::T_DK + c, r);
+          tmem_wait_ld();
+          float gk[32];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dk_row + c + e) = make_float4(g[e], g[e + 1], g[e + 2], g[e + 3]);
+          for (int e = 0; e < 32; ++e) gk[e] = __uint_as_float(r[e]);
+          if (p.rbf) {
+            // - k_j * sum_i dS'_ij (k from the swizzled K tile: column c + e is 16-byte unit ((c+e)%64)/8 of box (c+e)/64)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int cc = c + 8 * u;
+              const uint4 w = *reinterpret_cast<const uint4*>(kt_s + (cc / 64) * (TB * 128) + t * 128 +
+                                                              ((((cc % 64) / 8) ^ (t & 7)) << 4));
+              const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                gk[8 * u + 2 * e] -= __uint_as_float(ws[e] << 16) * ds_rowsum;
+                gk[8 * u + 2 * e + 1] -= __uint_as_float(ws[e] & 0xFFFF0000u) * ds_rowsum;
+              }
+            }
+          }
+          if (row_ok) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dk_row + c + e) =
+                  make_float4(p.c_q * gk[e], p.c_q * gk[e + 1], p.c_q * gk[e + 2], p.c_q * gk[e + 3]);
+          }
         }
       }
     } else if (n_it == 0 && j < p.S) {
       // no query sees this key tile: its gradients are zero
-      float* dv_row = p.dv + (static_cast<size_t>(nh) * p.S + j) * EV;
-      float* dk_row = p.dk + (static_cast<size_t>(nh) * p.S + j) * E;
-      for (int c = 0; c < EV; ++c) dv_row[c] = 0.f;
-      for (int c = 0; c < E; ++c) dk_row[c] = 0.f;
+      if (g == 0)
+        for (int c = 0; c < EV; ++c) dv_row[c] = 0.f;
+      else
+        for (int c = 0; c < E; ++c) dk_row[c] = 0.f;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == W_ISSUER) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
 // D_i = dout_i . out_i (fp32), lse2_i = lse_i * log2e, both padded per head to Lp
-// rows (D = 0, lse2 = -inf past L), and the sink gradient -sum_i 2^(s2 - lse2_i) D_i.
+// rows, and the sink gradient -sum_i 2^(s2 - lse2_i) D_i.  Past L, and on rows
+// whose lse is -inf (they see no key and have no output), lse2 = +inf, so that
+// 2^(z2 - lse2) = 0 there without a test; D = 0 past L.
 // One warp per padded row.
 template <int EV>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ out,
@@ -487,7 +616,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
   if (i >= L) {
     if (lane == 0) {
       dsum[pr] = 0.f;
-      lse2[pr] = -INFINITY;
+      lse2[pr] = INFINITY;
     }
     return;
   }
@@ -504,7 +633,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
   if (lane == 0) {
     const float l = lse[r];
     dsum[pr] = acc;
-    lse2[pr] = l * LOG2E;
+    lse2[pr] = l == -INFINITY ? INFINITY : l * LOG2E;
     if (sink != nullptr && dsink != nullptr) {  // a caller may pass sink logits without asking for dsink
       const int hq = static_cast<int>(head % Hq);
       if (l != -INFINITY) atomicAdd(dsink + hq, -ex2((sink[hq] - l) * LOG2E) * acc);
@@ -528,8 +657,8 @@ int launch_bwd_impl(const BwdArgs& a, float* ws, cudaStream_t stream) {
       a.dsink, a.Hq, a.L, Lp, prows);
   if (cudaGetLastError() != cudaSuccess) return -13;
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_map_rows(&tq, a.q, E, a.L, static_cast<long long>(a.N) * a.Hq, TB)) return -13;
-  if (!make_map_rows(&tdo, a.dout, EV, a.L, static_cast<long long>(a.N) * a.Hq, TB)) return -13;
+  if (!make_map_rows(&tq, a.q, E, a.L, static_cast<long long>(a.N) * a.Hq, QT)) return -13;
+  if (!make_map_rows(&tdo, a.dout, EV, a.L, static_cast<long long>(a.N) * a.Hq, QT)) return -13;
   if (!make_map_rows(&tk, a.k, E, a.S, static_cast<long long>(a.N) * a.H, TB)) return -13;
   if (!make_map_rows(&tv, a.v, EV, a.S, static_cast<long long>(a.N) * a.H, TB)) return -13;
   BwdParams p{};

@@ -56,8 +56,10 @@ constexpr int TB = 128;           // keys per CTA tile
 constexpr int QT = 64;            // queries per query tile
 constexpr int N_COMPUTE = 256;    // two warpgroups
 constexpr int W_DQ = N_COMPUTE / 32;  // first dQ readout warp
-constexpr int W_PRODUCER = W_DQ + 4, W_ISSUER = W_PRODUCER + 1;
-constexpr int BTHREADS = (W_ISSUER + 1) * 32;
+constexpr int W_PRODUCER = W_DQ + 4;
+constexpr int W_ISSUER = W_PRODUCER + 1;   // dP^T and dQ^T: the MMAs a warpgroup waits for
+constexpr int W_ISSUER2 = W_ISSUER + 1;    // S^T, dV and dK: the MMAs with slack
+constexpr int BTHREADS = (W_ISSUER2 + 1) * 32;
 
 // tcgen05 instruction descriptor with the A major bit as well (bit 15: MN-major A)
 __host__ __device__ constexpr uint32_t idesc_ab(uint32_t M, uint32_t N, uint32_t a_mn, uint32_t b_mn) {
@@ -71,20 +73,22 @@ struct BCfg {
   static constexpr int Q_BYTES = QT * E * 2;
   static constexpr int DO_BYTES = QT * EV * 2;
   static constexpr int LD_BYTES = 2 * QT * 4;                          // lse2 and D of the tile
-  static constexpr int NSTAGE = 4;
+  static constexpr int NSTAGE = 3;
   static constexpr int DS_BYTES = TB * QT * 2;                         // one dS'^T buffer
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + K_BYTES;
   static constexpr int OFF_Q = OFF_V + V_BYTES;                        // [NSTAGE] Q tiles
   static constexpr int OFF_DO = OFF_Q + NSTAGE * Q_BYTES;              // [NSTAGE] dO tiles
   static constexpr int OFF_DS = OFF_DO + NSTAGE * DO_BYTES;            // [2] dS'^T
-  static constexpr int OFF_LD = OFF_DS + 2 * DS_BYTES;                 // [NSTAGE] lse2[64], D[64]
+  static constexpr int OFF_DQS = OFF_DS + 2 * DS_BYTES;                // dQ staging, [64 queries][E] fp32
+  static constexpr int DQS_BYTES = QT * E * 4;
+  static constexpr int OFF_LD = OFF_DQS + DQS_BYTES;                   // [NSTAGE] lse2[64], D[64]
   static constexpr int OFF_BAR = OFF_LD + NSTAGE * LD_BYTES;
   // barriers
   static constexpr int B_KV = 0, B_QFULL = 1, B_QEMPTY = 1 + NSTAGE, B_SFULL = 1 + 2 * NSTAGE;
-  static constexpr int B_PFULL = B_SFULL + 2, B_DQFULL = B_SFULL + 4, B_DQEMPTY = B_SFULL + 6;
-  static constexpr int B_DKV = B_SFULL + 8, B_DRAIN = B_SFULL + 9;
-  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int B_PFULL = B_SFULL + 2, B_DQFULL = B_SFULL + 4;
+  static constexpr int B_DKV = B_SFULL + 6, B_DRAIN = B_SFULL + 7;  // B_DRAIN: [3], one per issuing thread
+  static constexpr int NBAR = B_DRAIN + 3;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -124,12 +128,36 @@ __device__ __forceinline__ bool bwait(uint32_t bar, uint32_t parity, volatile in
   return false;
 }
 
-__device__ __forceinline__ void red_add_f32(float* addr, float a) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
+// the two compute warpgroups only (named barrier 1); the dQ readout warpgroup only (named barrier 2)
+__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(N_COMPUTE) : "memory"); }
+__device__ __forceinline__ void dq_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+// the same barrier returning the AND of every thread's flag (a uniform decision)
+__device__ __forceinline__ bool dq_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 2, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
 }
 
-// the two compute warpgroups only (named barrier 1)
-__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(N_COMPUTE) : "memory"); }
+// Bulk tensor reduce-add (fp32, tile mode, no multicast) of a shared-memory box into global
+// memory at coordinates (c0, c1, c2); elements outside the tensor are skipped.
+__device__ __forceinline__ void bulk_reduce_add_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// every committed bulk operation of this thread has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed bulk operation of this thread has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -207,7 +235,7 @@ template <int E, int EV, bool MX>
 __global__ void __launch_bounds__(BTHREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const BwdParams p) {
+               const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BCfg<E, EV>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sb = smem_u32(smem_raw);
@@ -218,6 +246,7 @@ __global__ void __launch_bounds__(BTHREADS, 1)
   uint8_t* sp = smem_raw;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + C::OFF_MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + C::OFF_MISC + 4);
+  volatile int* dq_issued = reinterpret_cast<volatile int*>(sp + C::OFF_MISC + 8);  // tiles whose dQ^T is issued
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8u * i; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -245,19 +274,19 @@ __global__ void __launch_bounds__(BTHREADS, 1)
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
+    *dq_issued = 0;
     mbar_init(bar(C::B_KV), 1);
     for (int s = 0; s < C::NSTAGE; ++s) {
       mbar_init(bar(C::B_QFULL + s), 1);
-      mbar_init(bar(C::B_QEMPTY + s), 1);
+      mbar_init(bar(C::B_QEMPTY + s), 2);  // after dP^T (dQ readout warpgroup) and after dK (second issuer)
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(C::B_SFULL + b), 1);
+      mbar_init(bar(C::B_SFULL + b), 2);  // S^T (second issuer) and dP^T (dQ readout warpgroup)
       mbar_init(bar(C::B_PFULL + b), N_COMPUTE);
       mbar_init(bar(C::B_DQFULL + b), 1);
-      mbar_init(bar(C::B_DQEMPTY + b), 128);
     }
     mbar_init(bar(C::B_DKV), 1);
-    mbar_init(bar(C::B_DRAIN), 1);
+    for (int d = 0; d < 3; ++d) mbar_init(bar(C::B_DRAIN + d), 1);
     fence_barrier_init();
   }
   if (warp == W_ISSUER) {
@@ -300,136 +329,171 @@ __global__ void __launch_bounds__(BTHREADS, 1)
       for (int it = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); it < issued; ++it)
         mbar_wait(bar(C::B_QFULL + it % C::NSTAGE), (it / C::NSTAGE) & 1);
     }
-  } else if (warp == W_ISSUER) {
-    // ================= tcgen05 issuer =================
+  } else if (warp == W_ISSUER || warp == W_ISSUER2) {
+    // ================= tcgen05 issuers =================
+    // Three threads issue into the one in-order tensor pipe, so that an MMA a warpgroup waits
+    // for is never held up behind another thread's blocked issue: the first issuer sends dQ^T
+    // as soon as a tile's scores are consumed, the dQ readout warpgroup sends the dP^T that
+    // reuses the columns it has just read, and the second issuer sends S^T, dV and dK.  A
+    // commit covers its own thread's MMAs only: SFULL and QEMPTY take one commit from each of
+    // their two issuers.
     if (lane == 0) {
+      const bool urgent = warp == W_ISSUER;
       bool ok = bwait(bar(C::B_KV), 0, abort_flag);
       tc_fence_after();
       constexpr uint32_t hi = desc_hi_sw128(1024);
       const uint32_t k_lo_kmaj = desc_lo(sb + C::OFF_K, 16);
-      const uint32_t v_lo_kmaj = desc_lo(sb + C::OFF_V, 16);
       const uint32_t k_lo_mn = desc_lo(sb + C::OFF_K, TB * 128);
-      // K-major operands step 16 along K inside 64-column boxes (of 128 key rows or 64 query rows)
-      auto koff = [](int kk, int box_bytes) -> uint32_t {
-        return static_cast<uint32_t>(((kk / 4) * box_bytes + (kk % 4) * 32) >> 4);
-      };
-      // S^T and dP^T of tile it into S_b / DP_b
-      auto issue_s = [&](int it) {
-        const uint32_t q_lo = desc_lo(sb + C::OFF_Q + (it % C::NSTAGE) * C::Q_BYTES, 16);
-        const uint32_t d = tmem + C::T_S + 64 * (it & 1);
-#pragma unroll
-        for (int kk = 0; kk < E / 16; ++kk)
-          mma_ss_h(d, k_lo_kmaj + koff(kk, TB * 128), hi, q_lo + koff(kk, QT * 128), hi, C::IDESC_S, kk > 0 ? 1u : 0u);
-      };
-      auto issue_dp = [&](int it) {
-        const uint32_t do_lo = desc_lo(sb + C::OFF_DO + (it % C::NSTAGE) * C::DO_BYTES, 16);
-        const uint32_t d = tmem + C::T_DP + 64 * (it & 1);
-#pragma unroll
-        for (int kk = 0; kk < EV / 16; ++kk)
-          mma_ss_h(d, v_lo_kmaj + koff(kk, TB * 128), hi, do_lo + koff(kk, QT * 128), hi, C::IDESC_S,
-                   kk > 0 ? 1u : 0u);
-      };
-      // the rest of tile it once its scores are consumed: dQ^T into DP_b, dV, dK
-      auto issue_grads = [&](int it) {
-        const int b = it & 1, s = it % C::NSTAGE;
-        const uint32_t ds_base = sb + C::OFF_DS + b * C::DS_BYTES;
-        const uint32_t ds_lo_mn = desc_lo(ds_base, C::DS_BYTES);  // one 64-query box: the MN stride is unused
-        const uint32_t ds_lo_kmaj = desc_lo(ds_base, 16);
-#pragma unroll
-        for (int kk = 0; kk < TB / 16; ++kk)
-          mma_ss_h(tmem + C::T_DP + 64 * b, k_lo_mn + kk * 128, hi, ds_lo_mn + kk * 128, hi, C::IDESC_DQ,
-                   kk > 0 ? 1u : 0u);
-        mma_commit(bar(C::B_DQFULL + b));
-        // dV += P^T dO: query q's bf16 pair sits in column 64 b + 32 (q / 32) + (q % 32) / 2
-        const uint32_t do_lo_mn = desc_lo(sb + C::OFF_DO + s * C::DO_BYTES, QT * 128);
-        const uint32_t q_lo_mn = desc_lo(sb + C::OFF_Q + s * C::Q_BYTES, QT * 128);
-#pragma unroll
-        for (int kk = 0; kk < QT / 16; ++kk)
-          mma_ts_h(tmem + C::T_DV, tmem + C::T_S + 64 * b + 32 * (kk / 2) + 8 * (kk % 2), do_lo_mn + kk * 128, hi,
-                   C::IDESC_DV, (it > 0 || kk > 0) ? 1u : 0u);
-        // dK += dS'^T Q (A K-major over the tile's 64 queries: 32 bytes per step)
-#pragma unroll
-        for (int kk = 0; kk < QT / 16; ++kk)
-          mma_ss_h(tmem + C::T_DK, ds_lo_kmaj + kk * 2, hi, q_lo_mn + kk * 128, hi, C::IDESC_DK,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar(C::B_QEMPTY + s));  // Q, dO, lse2 and D of this stage are no longer read
-      };
-      // tiles 0 and 1 start at once (their buffers are fresh)
-      for (int it = 0; ok && it < 2 && it < n_it; ++it) {
-        ok = bwait(bar(C::B_QFULL + it % C::NSTAGE), (it / C::NSTAGE) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        issue_s(it);
-        issue_dp(it);
-        mma_commit(bar(C::B_SFULL + (it & 1)));
-      }
-      // Two event streams, served as they come: PFULL(np) (tile np's scores consumed) and
-      // DQEMPTY of tile ndp - 2 (DP_b free again for dP^T of tile ndp).
-      int np = 0, ndp = 2;
-      long long t_last = clock64();
-      while (ok && np < n_it) {
-        bool progress = false;
-        if (ndp < n_it && ndp - 2 < np && mbar_test(bar(C::B_DQEMPTY + (ndp & 1)), ((ndp - 2) >> 1) & 1)) {
+      if (urgent) {
+        // dQ^T = K^T dS'^T of tile it into DP_b once its scores are consumed (PFULL)
+        for (int it = 0; ok && it < n_it; ++it) {
+          const int b = it & 1;
+          if (!bwait(bar(C::B_PFULL + b), (it >> 1) & 1, abort_flag)) break;
           tc_fence_after();
-          issue_dp(ndp);  // S^T of tile ndp went out with the gradients of tile ndp - 2
-          mma_commit(bar(C::B_SFULL + (ndp & 1)));
-          ++ndp;
-          progress = true;
+          const uint32_t ds_lo_mn = desc_lo(sb + C::OFF_DS + b * C::DS_BYTES, C::DS_BYTES);  // one 64-query box
+#pragma unroll
+          for (int kk = 0; kk < TB / 16; ++kk)
+            mma_ss_h(tmem + C::T_DP + 64 * b, k_lo_mn + kk * 128, hi, ds_lo_mn + kk * 128, hi, C::IDESC_DQ,
+                     kk > 0 ? 1u : 0u);
+          mma_commit(bar(C::B_DQFULL + b));
+          *dq_issued = it + 1;  // the second issuer's dV and dK of the tile queue behind its dQ^T
         }
-        if (mbar_test(bar(C::B_PFULL + (np & 1)), (np >> 1) & 1)) {
-          tc_fence_after();
-          issue_grads(np);
-          if (np + 2 < n_it) {
-            if (!bwait(bar(C::B_QFULL + (np + 2) % C::NSTAGE), ((np + 2) / C::NSTAGE) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
+      } else {
+        // K-major operands step 16 along K inside 64-column boxes (of 128 key rows or 64 query rows)
+        auto koff = [](int kk, int box_bytes) -> uint32_t {
+          return static_cast<uint32_t>(((kk / 4) * box_bytes + (kk % 4) * 32) >> 4);
+        };
+        int n0 = 0, n1 = 0;  // next dV/dK, next S^T
+        long long t_last = clock64();
+        while (ok && n0 < n_it) {
+          bool progress = false;
+          // dV += P^T dO and dK += dS'^T Q of tile n0 once its scores are consumed and its dQ^T is
+          // issued (its own PFULL test orders this thread after the compute warpgroups' writes)
+          if (n0 < n1 && n0 < *dq_issued && mbar_test(bar(C::B_PFULL + (n0 & 1)), (n0 >> 1) & 1)) {
             tc_fence_after();
-            issue_s(np + 2);  // after the dV MMA that reads P^T in these columns
+            const int b = n0 & 1, st = n0 % C::NSTAGE;
+            const uint32_t do_lo_mn = desc_lo(sb + C::OFF_DO + st * C::DO_BYTES, QT * 128);
+            const uint32_t q_lo_mn = desc_lo(sb + C::OFF_Q + st * C::Q_BYTES, QT * 128);
+            const uint32_t ds_lo_kmaj = desc_lo(sb + C::OFF_DS + b * C::DS_BYTES, 16);
+            // query q's bf16 pair of P^T sits in column 64 b + 32 (q / 32) + (q % 32) / 2
+#pragma unroll
+            for (int kk = 0; kk < QT / 16; ++kk)
+              mma_ts_h(tmem + C::T_DV, tmem + C::T_S + 64 * b + 32 * (kk / 2) + 8 * (kk % 2), do_lo_mn + kk * 128,
+                       hi, C::IDESC_DV, (n0 > 0 || kk > 0) ? 1u : 0u);
+            // A = dS'^T K-major over the tile's 64 queries: 32 bytes per step
+#pragma unroll
+            for (int kk = 0; kk < QT / 16; ++kk)
+              mma_ss_h(tmem + C::T_DK, ds_lo_kmaj + kk * 2, hi, q_lo_mn + kk * 128, hi, C::IDESC_DK,
+                       (n0 > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bar(C::B_QEMPTY + st));  // Q, dO, lse2 and D of this stage are no longer read here
+            ++n0;
+            progress = true;
           }
-          ++np;
-          progress = true;
+          // S^T = K Q^T of tile n1 into S_b once Q landed and dV of tile n1 - 2 (reading P^T there) is issued
+          if (n1 < n_it && n1 - 2 < n0 && mbar_test(bar(C::B_QFULL + n1 % C::NSTAGE), (n1 / C::NSTAGE) & 1)) {
+            tc_fence_after();
+            const uint32_t q_lo = desc_lo(sb + C::OFF_Q + (n1 % C::NSTAGE) * C::Q_BYTES, 16);
+#pragma unroll
+            for (int kk = 0; kk < E / 16; ++kk)
+              mma_ss_h(tmem + C::T_S + 64 * (n1 & 1), k_lo_kmaj + koff(kk, TB * 128), hi, q_lo + koff(kk, QT * 128),
+                       hi, C::IDESC_S, kk > 0 ? 1u : 0u);
+            mma_commit(bar(C::B_SFULL + (n1 & 1)));
+            ++n1;
+            progress = true;
+          }
+          if (progress) {
+            t_last = clock64();
+          } else if (*abort_flag) {
+            ok = false;
+          } else if (clock64() - t_last > WAIT_LIMIT_CYCLES) {
+            record_timeout();
+            *abort_flag = 1;
+            ok = false;
+          }
         }
-        if (progress) {
-          t_last = clock64();
-        } else if (*abort_flag) {
-          ok = false;
-        } else if (clock64() - t_last > WAIT_LIMIT_CYCLES) {
-          record_timeout();
-          *abort_flag = 1;
-          ok = false;
-        }
+        mma_commit(bar(C::B_DKV));  // dV and dK are this thread's
       }
-      mma_commit(bar(C::B_DKV));
-      mma_commit(bar(C::B_DRAIN));
-      mbar_wait(bar(C::B_DRAIN), 0);
+      const uint32_t drain = bar(C::B_DRAIN + (urgent ? 0 : 1));
+      mma_commit(drain);
+      mbar_wait(drain, 0);
     }
   } else if (warp >= W_DQ) {
     // ================= dQ^T readout: lane = head-dimension index, column = query =================
-    const int t = threadIdx.x & 127;
+    // TMEM -> registers; the elected thread then sends dP^T of tile it + 2 into the columns just
+    // read (with its commits on SFULL and QEMPTY), while the warpgroup writes the tile to
+    // shared memory as fp32 [query][E] for bulk tensor reduce-adds into dq (the tensor map
+    // skips the rows past L).
+    const int e = threadIdx.x - 32 * W_DQ;  // head-dimension index = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const bool has_rows = (warp & 3) * 32 < E;  // lanes >= E hold nothing (E = 64)
+    const bool elected = threadIdx.x == 32 * W_DQ;
+    float* stage = reinterpret_cast<float*>(sp + C::OFF_DQS);
+    constexpr uint32_t hi = desc_hi_sw128(1024);
+    const uint32_t v_lo_kmaj = desc_lo(sb + C::OFF_V, 16);
+    // dP^T = V dO^T of tile t into DP_b once its dO has landed; then this thread's reads of the stage are done
+    auto issue_dp = [&](int t) -> bool {
+      const int st = t % C::NSTAGE;
+      if (!bwait(bar(C::B_QFULL + st), (t / C::NSTAGE) & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t do_lo = desc_lo(sb + C::OFF_DO + st * C::DO_BYTES, 16);
+#pragma unroll
+      for (int kk = 0; kk < EV / 16; ++kk) {
+        const uint32_t ko = static_cast<uint32_t>(((kk / 4) * (TB * 128) + (kk % 4) * 32) >> 4);
+        const uint32_t kq = static_cast<uint32_t>(((kk / 4) * (QT * 128) + (kk % 4) * 32) >> 4);
+        mma_ss_h(tmem + C::T_DP + 64 * (t & 1), v_lo_kmaj + ko, hi, do_lo + kq, hi, C::IDESC_S, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(bar(C::B_SFULL + (t & 1)));
+      mma_commit(bar(C::B_QEMPTY + st));
+      return true;
+    };
+    bool issue_ok = true;  // the elected thread's own waits
+    if (elected) {
+      issue_ok = bwait(bar(C::B_KV), 0, abort_flag);
+      for (int t = 0; issue_ok && t < 2 && t < n_it; ++t) issue_ok = issue_dp(t);
+    }
     for (int it = 0; it < n_it; ++it) {
       const int b = it & 1;
-      if (!__all_sync(0xffffffffu, bwait(bar(C::B_DQFULL + b), (it >> 1) & 1, abort_flag))) break;
+      bool ready = bwait(bar(C::B_DQFULL + b), (it >> 1) & 1, abort_flag);
       tc_fence_after();
-      if (has_rows) {
-        const int q0 = tile_q0(it);
-        float* dq_col = p.dq + (tile_head(it) * p.L + q0) * E + t;
-        const int lim = p.L - q0;
-#pragma unroll 1
-        for (int ch = 0; ch < QT / 32; ++ch) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + C::T_DP + 64 * b + 32 * ch, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (32 * ch + e < lim)
-              red_add_f32(dq_col + static_cast<size_t>(32 * ch + e) * E, p.c_q * __uint_as_float(r[e]));
-        }
+      float v[QT];
+      if (has_rows && ready) {
+        tmem_ld32f<0>(tmem + lane_base + C::T_DP + 64 * b, v);
+        tmem_ld32f<32>(tmem + lane_base + C::T_DP + 64 * b + 32, v);
+        tmem_wait_ld();
       }
       tc_fence_before();
-      mbar_arrive(bar(C::B_DQEMPTY + b));
+      // every lane's loads of DP_b are complete; all four warps leave together on a failed wait
+      if (!dq_bar_and(ready && issue_ok)) break;
+      if (elected && it + 2 < n_it) {
+        tc_fence_after();
+        issue_ok = issue_dp(it + 2);
+      }
+      // two halves of 32 queries, each with its own bulk reduce issued by its own thread (lane 0
+      // of the first and second warp: two reduces in flight): a half is rewritten once the
+      // previous tile's reduce of the same half has read it
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const bool half_issuer = threadIdx.x == 32 * (W_DQ + h);
+        if (half_issuer) bulk_wait_read_all();
+        dq_bar();
+        if (has_rows) {
+#pragma unroll
+          for (int c = 0; c < QT / 2; ++c) stage[(32 * h + c) * E + e] = p.c_q * v[32 * h + c];
+        }
+        fence_proxy_async_smem();  // the staging half is read by the bulk copy (async proxy)
+        dq_bar();
+        if (half_issuer) {
+          bulk_reduce_add_3d(&tm_dq, sb + C::OFF_DQS + h * (QT / 2) * E * 4, 0, tile_q0(it) + 32 * h,
+                             static_cast<int>(tile_head(it)));
+          bulk_commit();
+        }
+      }
+    }
+    if (threadIdx.x == 32 * (W_DQ + 1)) bulk_wait_all();  // every reduce has completed before the CTA exits
+    if (elected) {
+      bulk_wait_all();
+      mma_commit(bar(C::B_DRAIN + 2));
+      mbar_wait(bar(C::B_DRAIN + 2), 0);
     }
   } else {
     // ================= compute warpgroups =================
@@ -506,7 +570,8 @@ __global__ void __launch_bounds__(BTHREADS, 1)
       }
       // P^T as bf16 pairs over S^T columns this warpgroup has already read
       tmem_st16(tmem + lane_base + C::T_S + 64 * b + 32 * g, pk);
-      // dS'^T row t of buffer b: this warpgroup's queries are 16-byte units 4 g .. 4 g + 3
+      // dS'^T row t of buffer b: this warpgroup's queries are 16-byte units 4 g .. 4 g + 3 (SFULL
+      // implies that dK and dQ^T of tile it - 2 have read the buffer)
       uint8_t* ds_row = sp + C::OFF_DS + b * C::DS_BYTES + t * 128;
 #pragma unroll
       for (int v = 0; v < 4; ++v)
@@ -641,6 +706,24 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
   }
 }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// fp32 dq [heads, L, E] with an E x 32 x 1 box, no swizzle (each staging half is dense
+// [32 queries][E]); reduces into rows past L are dropped by the tensor map.
+bool make_map_dq(CUtensorMap* map, float* dq, int E, long long L, long long heads) {
+  auto fn = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
+  if (!fn) return false;
+  cuuint64_t gdim[3] = {static_cast<cuuint64_t>(E), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(heads)};
+  cuuint64_t gstride[2] = {static_cast<cuuint64_t>(E) * 4, static_cast<cuuint64_t>(L) * E * 4};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(E), static_cast<cuuint32_t>(QT / 2), 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dq, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 template <int E, int EV>
 int launch_bwd_impl(const BwdArgs& a, float* ws, cudaStream_t stream) {
   using C = BCfg<E, EV>;
@@ -661,6 +744,8 @@ int launch_bwd_impl(const BwdArgs& a, float* ws, cudaStream_t stream) {
   if (!make_map_rows(&tdo, a.dout, EV, a.L, static_cast<long long>(a.N) * a.Hq, QT)) return -13;
   if (!make_map_rows(&tk, a.k, E, a.S, static_cast<long long>(a.N) * a.H, TB)) return -13;
   if (!make_map_rows(&tv, a.v, EV, a.S, static_cast<long long>(a.N) * a.H, TB)) return -13;
+  CUtensorMap tdq;
+  if (!make_map_dq(&tdq, a.dq, E, a.L, static_cast<long long>(a.N) * a.Hq)) return -13;
   BwdParams p{};
   p.lse2 = lse2;
   p.dsum = dsum;
@@ -691,7 +776,7 @@ int launch_bwd_impl(const BwdArgs& a, float* ws, cudaStream_t stream) {
     return -13;
   const long long grid = static_cast<long long>(a.N) * a.H * ((a.S + TB - 1) / TB);
   if (grid > 0x7fffffffLL) return -2;
-  kern<<<static_cast<unsigned>(grid), BTHREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+  kern<<<static_cast<unsigned>(grid), BTHREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError() == cudaSuccess ? 0 : -13;
 }
 

@@ -77,6 +77,12 @@ CASES = [
     R("b_rbf_window_keep_both_pads_450", L=450, S=450, N=2, mode="rbf", mask_kind="window", window=100,
       keep_mask="random10", pad_left=0.3, pad_right=0.3, scale=0.05),
     R("b_keep_right_pad_L200_S700", L=200, S=700, N=2, keep_mask="random10", pad_right=0.5, Ev=128),
+    # every key tile walks exactly one, two or three 64-query tiles (pipeline fill and drain with
+    # the dK of a tile issued out of order)
+    R("b_dot_none_64_one_tile_e128", L=64, S=64, E=128, Ev=128, Hq=1, H=1),
+    R("b_dot_none_128_two_tiles_e128", L=128, S=128, E=128, Ev=128, Hq=1, H=1),
+    R("b_dot_none_192_three_tiles_e128", L=192, S=192, E=128, Ev=128, Hq=1, H=1),
+    R("b_rbf_none_160_three_tiles_ragged", L=160, S=160, mode="rbf", Hq=1, H=1, scale=0.05),
 ]
 
 

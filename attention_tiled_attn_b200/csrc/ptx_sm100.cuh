@@ -204,6 +204,24 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// The same load with the 32 columns landing as floats in z[B .. B+31] (no copy
+// from an integer staging array).
+template <int B, int N>
+__device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float (&z)[N]) {
+  static_assert(B + 32 <= N, "tmem_ld32f range");
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=f"(z[B + 0]), "=f"(z[B + 1]), "=f"(z[B + 2]), "=f"(z[B + 3]), "=f"(z[B + 4]), "=f"(z[B + 5]),
+        "=f"(z[B + 6]), "=f"(z[B + 7]), "=f"(z[B + 8]), "=f"(z[B + 9]), "=f"(z[B + 10]), "=f"(z[B + 11]),
+        "=f"(z[B + 12]), "=f"(z[B + 13]), "=f"(z[B + 14]), "=f"(z[B + 15]), "=f"(z[B + 16]), "=f"(z[B + 17]),
+        "=f"(z[B + 18]), "=f"(z[B + 19]), "=f"(z[B + 20]), "=f"(z[B + 21]), "=f"(z[B + 22]), "=f"(z[B + 23]),
+        "=f"(z[B + 24]), "=f"(z[B + 25]), "=f"(z[B + 26]), "=f"(z[B + 27]), "=f"(z[B + 28]), "=f"(z[B + 29]),
+        "=f"(z[B + 30]), "=f"(z[B + 31])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -354,14 +372,6 @@ __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
       "mov.b64 {%0, %1}, rd;\n\t}"
       : "+f"(d0), "+f"(d1)
       : "f"(a0), "f"(a1));
-}
-
-// 32-byte global store (sm_100); the address must be 32-byte aligned
-__device__ __forceinline__ void st_global_v8(void* ptr, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
-                                             uint32_t a5, uint32_t a6, uint32_t a7) {
-  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(a0), "r"(a1), "r"(a2),
-               "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
-               : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

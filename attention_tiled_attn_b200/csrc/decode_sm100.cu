@@ -327,8 +327,7 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int last_phase[C::NSTAGE];
-      for (int s = 0; s < C::NSTAGE; ++s) last_phase[s] = -1;
+      int issued = 0;
       for (long long c = c_begin; c < c_end; ++c) {
         const int idx = static_cast<int>(c - c_begin);
         const int s = idx % C::NSTAGE;
@@ -346,10 +345,11 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
           tma_load_3d(dst + b * (DC * 128), &tm_k, full_bar(s), b * 64, key0, static_cast<int>(u));
         for (int b = 0; b < EV / 64; ++b)
           tma_load_3d(dst + E * DC * 2 + b * (DC * 128), &tm_v, full_bar(s), b * 64, key0, static_cast<int>(u));
-        last_phase[s] = ph;
+        issued = idx + 1;
       }
-      for (int s = 0; s < C::NSTAGE; ++s)
-        if (last_phase[s] >= 0) mbar_wait(full_bar(s), last_phase[s]);
+      // drain: the last NSTAGE copies (one per stage) have landed before exit
+      for (int idx = issued > C::NSTAGE ? issued - C::NSTAGE : 0; idx < issued; ++idx)
+        mbar_wait(full_bar(idx % C::NSTAGE), (idx / C::NSTAGE) & 1);
     }
     return;
   }

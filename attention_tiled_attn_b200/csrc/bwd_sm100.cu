@@ -665,7 +665,9 @@ __global__ void __launch_bounds__(BTHREADS, 1)
 // rows, and the sink gradient -sum_i 2^(s2 - lse2_i) D_i.  Past L, and on rows
 // whose lse is -inf (they see no key and have no output), lse2 = +inf, so that
 // 2^(z2 - lse2) = 0 there without a test; D = 0 past L.
-// One warp per padded row.
+// A row takes EV / 8 lanes, each reading 16 bytes of out and of dout; a warp covers
+// 256 / EV rows of one head (Lp is a multiple of 128), so the sink gradient is
+// summed over the warp before its one atomic.
 template <int EV>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ out,
                                                       const __nv_bfloat16* __restrict__ dout,
@@ -673,36 +675,46 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
                                                       float* __restrict__ dsum, float* __restrict__ lse2,
                                                       float* __restrict__ dsink, int Hq, int L, int Lp,
                                                       long long prows) {
-  const long long pr = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  constexpr int LPR = EV / 8;        // lanes per row
+  constexpr int RPW = 32 / LPR;      // rows per warp
   const int lane = threadIdx.x & 31;
-  if (pr >= prows) return;
-  const long long head = pr / Lp;
-  const int i = static_cast<int>(pr % Lp);
-  if (i >= L) {
-    if (lane == 0) {
-      dsum[pr] = 0.f;
-      lse2[pr] = INFINITY;
-    }
-    return;
-  }
-  const long long r = head * L + i;
+  const long long pr = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * RPW + lane / LPR;
+  const int sub = lane % LPR;
+  const bool row_in = pr < prows;
+  const long long head = row_in ? pr / Lp : 0;
+  const int i = row_in ? static_cast<int>(pr % Lp) : 0;
+  const bool live = row_in && i < L;
   float acc = 0.f;
-  for (int e = lane * 2; e < EV; e += 64) {
-    const __nv_bfloat162 o2 = *reinterpret_cast<const __nv_bfloat162*>(out + r * EV + e);
-    const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162*>(dout + r * EV + e);
-    acc = fmaf(__low2float(o2), __low2float(d2), acc);
-    acc = fmaf(__high2float(o2), __high2float(d2), acc);
+  if (live) {
+    const long long r = head * L + i;
+    const uint4 o4 = *reinterpret_cast<const uint4*>(out + r * EV + sub * 8);
+    const uint4 d4 = *reinterpret_cast<const uint4*>(dout + r * EV + sub * 8);
+    const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w}, dw[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc = fmaf(__uint_as_float(ow[e] << 16), __uint_as_float(dw[e] << 16), acc);
+      acc = fmaf(__uint_as_float(ow[e] & 0xFFFF0000u), __uint_as_float(dw[e] & 0xFFFF0000u), acc);
+    }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane == 0) {
-    const float l = lse[r];
-    dsum[pr] = acc;
-    lse2[pr] = l == -INFINITY ? INFINITY : l * LOG2E;
-    if (sink != nullptr && dsink != nullptr) {  // a caller may pass sink logits without asking for dsink
-      const int hq = static_cast<int>(head % Hq);
-      if (l != -INFINITY) atomicAdd(dsink + hq, -ex2((sink[hq] - l) * LOG2E) * acc);
+  for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  float g = 0.f;  // this row's sink-gradient term
+  if (row_in && sub == 0) {
+    if (!live) {
+      dsum[pr] = 0.f;
+      lse2[pr] = INFINITY;
+    } else {
+      const float l = lse[head * L + i];
+      dsum[pr] = acc;
+      lse2[pr] = l == -INFINITY ? INFINITY : l * LOG2E;
+      if (sink != nullptr && l != -INFINITY) g = -ex2((sink[head % Hq] - l) * LOG2E) * acc;
     }
+  }
+  if (sink != nullptr && dsink != nullptr) {  // a caller may pass sink logits without asking for dsink
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) g += __shfl_xor_sync(0xffffffffu, g, o);
+    const long long pr0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * RPW;
+    if (lane == 0 && pr0 < prows && g != 0.f) atomicAdd(dsink + (pr0 / Lp) % Hq, g);
   }
 }
 
@@ -735,7 +747,8 @@ int launch_bwd_impl(const BwdArgs& a, float* ws, cudaStream_t stream) {
   if (cudaMemsetAsync(a.dq, 0, static_cast<size_t>(rows) * E * sizeof(float), stream) != cudaSuccess) return -13;
   if (a.dsink && cudaMemsetAsync(a.dsink, 0, static_cast<size_t>(a.Hq) * sizeof(float), stream) != cudaSuccess)
     return -13;
-  bwd_pre_kernel<EV><<<static_cast<unsigned>((prows + 7) / 8), 256, 0, stream>>>(
+  constexpr long long ROWS_PER_BLOCK = 8 * (256 / EV);
+  bwd_pre_kernel<EV><<<static_cast<unsigned>((prows + ROWS_PER_BLOCK - 1) / ROWS_PER_BLOCK), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(a.out), static_cast<const __nv_bfloat16*>(a.dout), a.lse, a.sink, dsum, lse2,
       a.dsink, a.Hq, a.L, Lp, prows);
   if (cudaGetLastError() != cudaSuccess) return -13;

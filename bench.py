@@ -49,13 +49,16 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FFMA_PER_CLK_SM = 122
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
-# dominant kernel from one ncu capture of the same kernel build; the capture
-# command and counters are in profiles/.  Must be reset when the kernel changes.
+# dominant kernel from one ncu capture of the same kernel build, with the batch N
+# of that capture; the traffic of these kernels grows in proportion to N, so a
+# line at another N reports it scaled.  The capture command and counters are in
+# profiles/.  Must be reset when the kernel changes.  Keyed by the line's label:
+# a variant line (another mask, mode or key selection) has no entry, so null.
 NCU_TRAFFIC_BYTES = {
-    "dot_causal_2k_bf16": 132_508_416 + 11_135_232,          # prefill_kernel<128,128,dot> (plain variant)
-    # decode_partial_kernel<128,128> with the fused combine: batch-2 capture scaled by 16 to batch 32
-    "decode_sink_gqa_128k_bf16": 16 * (1_073_872_128 + 6_788_096),
-    "dot_causal_2k_bf16:backward": 453_322_496 + 293_284_608,  # bwd_kernel<128,128> (--backward)
+    "dot_causal_2k_bf16": (132_508_416 + 11_135_232, 4),          # prefill_kernel<128,128,dot> (plain variant)
+    "dot_causal_2k_bf16:backward": (453_969_920 + 291_908_608, 4),  # bwd_kernel<128,128> (--backward)
+    # decode_partial_kernel<128,128> with the fused combine (a batch-2 capture: 16 GB of cache at batch 32)
+    "decode_sink_gqa_128k_bf16": (1_073_880_576 + 3_166_976, 2),
 }
 
 
@@ -279,7 +282,7 @@ def time_device(fn, steps, warmup, flush_buf, stream):
     return sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / 1e3
 
 
-def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=False):
+def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=False, label=None):
     import torch
 
     import attention_tiled_attn_b200 as attn
@@ -341,8 +344,11 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
     else:
         peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         punit = "GB/s"
-    key = name + (":backward" if r.backward else "") + (f":select{r.n_sel}" if r.n_sel > 0 else "")
-    traffic = NCU_TRAFFIC_BYTES.get(key)
+    key = label or (name + (":backward" if r.backward else "") + (f":select{r.n_sel}" if r.n_sel > 0 else ""))
+    traffic = None
+    if key in NCU_TRAFFIC_BYTES:
+        t_bytes, t_n = NCU_TRAFFIC_BYTES[key]
+        traffic = t_bytes * r.N // t_n
     res = {
         "recipe": r, "amount": amount, "unit": unit, "secs_max": secs_max, "secs": secs,
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": punit,
@@ -595,7 +601,7 @@ def ours(args):
             sw.RECIPES[rr.name] = rr
             try:
                 k = max(5, args.steps // 4)
-                res = run_workload(rr.name, k, args.warmup, pg, flush, peaks, peak_kind)
+                res = run_workload(rr.name, k, args.warmup, pg, flush, peaks, peak_kind, label=label)
             finally:
                 sw.RECIPES[rr.name] = base
             extra[label] = {

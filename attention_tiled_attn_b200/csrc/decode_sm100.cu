@@ -493,11 +493,13 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
     const int key0 = GATHER ? 0 : chunk_key0<STREAM>(p, static_cast<int>(c % p.nc)) + j0;
     const int* keys_c = reinterpret_cast<const int*>(sp + C::OFF_KEYS) + s * DC + j0;  // GATHER
 
-    // S = Q K^T for 16 keys (two n-tiles of 8).  RBF: the B fragments also give
-    // ||k||^2: lane l holds dimensions 2(l%4) + {0, 1, 8, 9} of each 16-wide slice
-    // for key l/4 of n-tile 0 (b0, b1) and of n-tile 1 (b2, b3)
+    // S = Q K^T for 16 keys (two n-tiles of 8).  Lane l holds dimensions
+    // 2(l%4) + {0, 1, 8, 9} of each 16-wide slice for key l/4 of n-tile 0 (b0, b1)
+    // and key 8 + l/4 of n-tile 1 (b2, b3).  RBF: in the order {b0, b2, b1, b3} the
+    // same registers are the A fragment of the 16 keys x 16 dimensions block, so two
+    // more MMAs accumulate the 16 x 16 Gram block K K^T, whose diagonal is ||k||^2
     float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    float kq0 = 0.f, kq1 = 0.f;  // partial squared norms of keys lane/4 and 8 + lane/4
+    float gram[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // keys x keys 0-7, keys x keys 8-15
     {
       const int mat = lane >> 3;
       const int krow = j0 + (mat >> 1) * 8 + (lane & 7);
@@ -508,29 +510,23 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
         mma16816(sc[0], qa[kk], b0, b1);
         mma16816(sc[1], qa[kk], b2, b3);
         if constexpr (RBF) {
-          const uint32_t wv[4] = {b0, b1, b2, b3};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float lo = __uint_as_float(wv[q] << 16), hi = __uint_as_float(wv[q] & 0xFFFF0000u);
-            float& acc = q < 2 ? kq0 : kq1;
-            acc = fmaf(lo, lo, fmaf(hi, hi, acc));
-          }
+          const uint32_t ka[4] = {b0, b2, b1, b3};
+          mma16816(gram[0], ka, b0, b1);
+          mma16816(gram[1], ka, b2, b3);
         }
       }
     }
-    // RBF: the four lanes of each key complete its norm; each lane then fetches the
-    // norms of the keys in its accumulator fragment (keys t*8 + cq + {0, 1})
+    // RBF: each lane fetches the norms of the keys in its accumulator fragment (keys
+    // t*8 + cq + {0, 1}).  Gram entry (i, i) of the first block sits in register i % 2 of
+    // lane 9 (i / 2) + 4 (i % 2); entry (8 + i, 8 + i) of the second in register 2 + i % 2
+    // of the same lane (the C fragment: lane 4g + u holds rows g, g + 8 and columns 2u, 2u + 1)
     float kn[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
     if constexpr (RBF) {
-      kq0 += __shfl_xor_sync(0xffffffffu, kq0, 1);
-      kq0 += __shfl_xor_sync(0xffffffffu, kq0, 2);
-      kq1 += __shfl_xor_sync(0xffffffffu, kq1, 1);
-      kq1 += __shfl_xor_sync(0xffffffffu, kq1, 2);
-#pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        kn[0][x] = __shfl_sync(0xffffffffu, kq0, 4 * (cq + x));
-        kn[1][x] = __shfl_sync(0xffffffffu, kq1, 4 * (cq + x));
-      }
+      const int src = 9 * (lane & 3);  // cq / 2 = lane % 4
+      kn[0][0] = __shfl_sync(0xffffffffu, gram[0][0], src);
+      kn[0][1] = __shfl_sync(0xffffffffu, gram[0][1], src + 4);
+      kn[1][0] = __shfl_sync(0xffffffffu, gram[1][2], src);
+      kn[1][1] = __shfl_sync(0xffffffffu, gram[1][3], src + 4);
     }
     // logits in base 2 (rbf: 2 scale q.k - scale ||k||^2), masks and bias
     const bool need_mask = GATHER || EXT || p.mask_kind != MASK_NONE || p.bias != nullptr || key0 + 16 > p.S;

@@ -363,8 +363,13 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
 
 
 def e2e_measure(res, steps, warmup):
-    """Same metric through the public API with pinned host buffers: every step
-    copies its inputs host->device, runs attn_fwd and reads the output back."""
+    """Same metric through the public API with pinned host buffers: every step copies
+    its inputs host->device, runs attn_fwd and reads the output back.  Steps are
+    pipelined the way a caller streaming batches would run them: the host->device
+    copies on one stream, the calls in order on another (they share the library's
+    workspace), the device->host copies on a third, with two device copies of the
+    inputs and outputs so that step k's input copy and step k-1's output copy overlap
+    step k-1's and step k's compute."""
     import torch
 
     import attention_tiled_attn_b200 as attn
@@ -374,39 +379,64 @@ def e2e_measure(res, steps, warmup):
         return e2e_backward(res, steps, warmup)
     names = ("q", "k", "v", "key_idx") if r.n_sel > 0 else ("q", "k", "v")
     host = {k: t[k].cpu().pin_memory() for k in names}
-    dev = {k: torch.empty_like(t[k]) for k in names}
-    out_host = torch.empty(res["out"].shape, dtype=res["out"].dtype).pin_memory()
-    lse_host = torch.empty(res["lse"].shape, dtype=torch.float32).pin_memory()
-    stream = torch.cuda.current_stream()
+    dev = [{k: torch.empty_like(t[k]) for k in names} for _ in range(2)]
+    outs = [(torch.empty_like(res["out"]), torch.empty_like(res["lse"])) for _ in range(2)]
+    out_host = [torch.empty(res["out"].shape, dtype=res["out"].dtype).pin_memory() for _ in range(2)]
+    lse_host = [torch.empty(res["lse"].shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     h2d = sum(host[k].numel() * host[k].element_size() for k in host)
-    d2h = out_host.numel() * out_host.element_size() + lse_host.numel() * 4
+    d2h = out_host[0].numel() * out_host[0].element_size() + lse_host[0].numel() * 4
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    ran = [None, None]   # compute of the step that last used buffer set i (its inputs may be overwritten after)
+    read = [None, None]  # output copy of the step that last used buffer set i (its outputs may be overwritten after)
 
-    def step():
-        for k in names:
-            dev[k].copy_(host[k], non_blocking=True)
-        if r.n_sel > 0:
-            attn.attn_decode_indexed(dev["q"], dev["k"], dev["v"], dev["key_idx"], scale=r.scale, sink=t["sink"],
-                                     mask_kind=r.mask_kind, window=r.window, bias=t["bias"], out=res["out"],
-                                     lse=res["lse"], stream=stream)
-        else:
-            attn.attn_fwd(dev["q"], dev["k"], dev["v"], scale=r.scale, mode=r.mode, sink=t["sink"],
-                          mask_kind=r.mask_kind, window=r.window, keep_first=r.keep, bias=t["bias"], out=res["out"],
-                          lse=res["lse"], stream=stream, mask_bits=t["mask_bits"], kv_start=t["kv_start"],
-                          kv_end=t["kv_end"])
-        out_host.copy_(res["out"], non_blocking=True)
-        lse_host.copy_(res["lse"], non_blocking=True)
+    def step(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if ran[b] is not None:
+                s_in.wait_event(ran[b])
+            for k in names:
+                dev[b][k].copy_(host[k], non_blocking=True)
+            landed = ev()
+            landed.record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(landed)
+            if read[b] is not None:
+                s_run.wait_event(read[b])
+            o, l = outs[b]
+            if r.n_sel > 0:
+                attn.attn_decode_indexed(dev[b]["q"], dev[b]["k"], dev[b]["v"], dev[b]["key_idx"], scale=r.scale,
+                                         sink=t["sink"], mask_kind=r.mask_kind, window=r.window, bias=t["bias"],
+                                         out=o, lse=l, stream=s_run)
+            else:
+                attn.attn_fwd(dev[b]["q"], dev[b]["k"], dev[b]["v"], scale=r.scale, mode=r.mode, sink=t["sink"],
+                              mask_kind=r.mask_kind, window=r.window, keep_first=r.keep, bias=t["bias"], out=o,
+                              lse=l, stream=s_run, mask_bits=t["mask_bits"], kv_start=t["kv_start"],
+                              kv_end=t["kv_end"])
+            ran[b] = ev()
+            ran[b].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ran[b])
+            out_host[b].copy_(o, non_blocking=True)
+            lse_host[b].copy_(l, non_blocking=True)
+            read[b] = ev()
+            read[b].record(s_out)
 
-    for _ in range(warmup):
-        step()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        step()
-    b.record(stream)
+    z = torch.cuda.Event(enable_timing=True)
+    a.record(s_in)
+    s_run.wait_event(a)
+    s_out.wait_event(a)
+    for i in range(steps):
+        step(i)
+    s_in.wait_stream(s_run)
+    s_in.wait_stream(s_out)
+    z.record(s_in)
     torch.cuda.synchronize()
-    secs = a.elapsed_time(b) / 1e3
+    secs = a.elapsed_time(z) / 1e3
     for k in list(host):
         del host[k]
     return {"value": round(rate(res["amount"], secs / steps, res["unit"]), 3), "unit": res["unit"],

@@ -355,7 +355,10 @@ def run_workload(name, steps, warmup, pg, flush_buf, peaks, peak_kind, clocks=Fa
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": ("derived: FFMA/clk/SM x 2 x SMs x max SM clock" if bound == "fma" else
                                      f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback")},
-        "launches_per_step": 2 if (is_decode(r) or r.backward) else 1,  # decode: partial + combine; backward: pre + main
+        # this library's kernels per step: backward = pre-pass + main; a bf16 prefill with a float
+        # bias = keep-bit pre-pass + prefill; decode (combine fused) and the rest = one
+        "launches_per_step": 2 if (r.backward or (r.bias != "none" and r.dtype == "bf16" and not is_decode(r)
+                                                   and r.n_sel == 0 and r.mask_kind != "streaming")) else 1,
         "clocks": sampler.summary() if sampler else None,
         "tensors": t, "out": out, "lse": lse, "dout": dout if r.backward else None,
     }

@@ -617,6 +617,9 @@ def ours(args):
                 runs.append((name + ":backward", dataclasses.replace(r0, backward=True)))
             if r0.sink != "none":
                 runs.append((name + ":no_sink_control", dataclasses.replace(r0, sink="none")))
+            # the backward of the sink + GQA window workload (a 64-wide head dimension, groups of 8)
+            if r0.mask_kind == "window" and not is_decode(r0):
+                runs.append((name + ":backward", dataclasses.replace(r0, backward=True)))
             # StreamingLLM variant: 4 kept initial tokens plus the window (decode: a 4096-key window)
             if r0.mask_kind == "window":
                 runs.append((name + ":streaming_keep4", dataclasses.replace(r0, mask_kind="streaming", keep=4)))

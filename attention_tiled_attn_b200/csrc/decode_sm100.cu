@@ -53,8 +53,13 @@ namespace attn {
 namespace {
 
 constexpr int DC = 64;             // keys per chunk
-constexpr int DWARPS = 4;          // consumer warps (16 keys each)
-constexpr int DTHREADS = (DWARPS + 1) * 32;
+constexpr int DWARPS = 4;          // consumer warps per group (16 keys of a chunk each)
+// Consumer groups: two groups of four warps take alternate chunks, so each SMSP runs two
+// consumer warps and one's dependency chains hide behind the other's (the listed-key
+// variant, with its four gathering warps, keeps one group).
+template <bool GATHER>
+__host__ __device__ constexpr int n_groups() { return GATHER ? 1 : 2; }
+constexpr int DTHREADS = (2 * DWARPS + 1) * 32;  // two consumer groups + the producer
 // GATHER: producer warps, each issuing every GWARPS-th copy instruction of a chunk.  One warp
 // keeps too few copies in flight for random rows; 4 measured best (5 and 6 were slower).
 constexpr int GWARPS = 4;
@@ -98,7 +103,12 @@ template <int E, int EV, bool GATHER = false>
 struct DCfg {
   static constexpr int K_BYTES = DC * E * 2;  // V part of a stage starts here
   static constexpr int STAGE_BYTES = DC * (E + EV) * 2;
-  static constexpr int NSTAGE = (E + EV >= 256) ? 5 : (GATHER ? 7 : 8);
+  // With two consumer groups taking alternate chunks the count is even, so stage s is
+  // always consumed by group s % 2: each full barrier then has one waiting group, which
+  // waits its phases in order (a group that waited on a stage shared with the other could
+  // ask for the phase after an incomplete one, and its parity test would pass early).
+  static constexpr int NSTAGE = (E + EV >= 256) ? (GATHER ? 5 : 6) : (GATHER ? 7 : 8);
+  static_assert(GATHER || NSTAGE % 2 == 0, "each stage belongs to one consumer group");
   static constexpr int OFF_STAGES = 0;
   static constexpr int OFF_MERGE = NSTAGE * STAGE_BYTES;              // [DWARPS][16][EV] f32
   static constexpr int OFF_ML = OFF_MERGE + DWARPS * 16 * EV * 4;     // [DWARPS][16][2] f32
@@ -151,7 +161,22 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-__device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(DWARPS * 32) : "memory"); }
+// every consumer warp (named barrier 1); the _and form returns the AND of the threads' flags
+template <int NT>
+__device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
+template <int NT>
+__device__ __forceinline__ bool consumer_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(NT)
+      : "memory");
+  return r != 0;
+}
 
 // byte offset of (row, 16-byte chunk c) inside a swizzled chunk buffer of 64-row, 128-byte boxes
 __device__ __forceinline__ uint32_t sw_off(int row, int c16) {
@@ -227,6 +252,8 @@ __device__ __forceinline__ void combine_row(const DecodeParams& p, long long u, 
 }
 
 template <int E, int EV, bool STREAM, bool GATHER, bool EXT, bool RBF>
+// 288 threads (256 for the listed-key variant): nine warps put three on one SMSP, whose
+// quarter of the register file (16384) caps a thread at 168 registers
 __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
     decode_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const DecodeParams p, const ExtraArgs ga) {
@@ -322,7 +349,10 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
     cp_async_wait_all();  // no copy may still be in flight at exit
     return;
   }
-  if (warp == DWARPS) {
+  constexpr int NGRP = n_groups<GATHER>();
+  constexpr int NCW = NGRP * DWARPS;  // consumer warps
+  constexpr int NCT = NCW * 32;       // consumer threads
+  if (warp == NCW) {
     // ---------------- producer ----------------
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
@@ -355,6 +385,8 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
   }
 
   // ---------------- consumers ----------------
+  const int grp = warp / DWARPS;  // consumer group: the chunks idx = c - c_begin with idx % NGRP == grp
+  const int wq = warp % DWARPS;   // this warp's 16 keys of each chunk
   const int rA = lane >> 2;       // fragment rows rA and rA + 8
   const int cq = (lane & 3) * 2;  // fragment column pair
   const int off = p.S - p.L;
@@ -374,7 +406,6 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
   uint32_t qa[E / 16][4];
   float o[EV / 8][4];
   float m_run[2], l_run[2];
-  long long cur_unit = -1;
   bool ok = true;
 
   auto load_q = [&](long long u) {
@@ -409,8 +440,8 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
   };
   float* merge_o = reinterpret_cast<float*>(sp + C::OFF_MERGE);
   float* merge_ml = reinterpret_cast<float*>(sp + C::OFF_ML);
-  auto flush = [&](long long u) {
-    // per-warp state -> shared memory
+  // this warp's state -> its slot wq of the shared merge buffer (l summed over the quad)
+  auto store_state = [&]() {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float l = l_run[h];
@@ -418,18 +449,49 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
       l += __shfl_xor_sync(0xffffffffu, l, 2);
       const int r = rA + 8 * h;
       if ((lane & 3) == 0) {
-        merge_ml[(warp * 16 + r) * 2 + 0] = m_run[h];
-        merge_ml[(warp * 16 + r) * 2 + 1] = l;
+        merge_ml[(wq * 16 + r) * 2 + 0] = m_run[h];
+        merge_ml[(wq * 16 + r) * 2 + 1] = l;
       }
 #pragma unroll
       for (int t = 0; t < EV / 8; ++t) {
-        merge_o[(warp * 16 + r) * EV + t * 8 + cq] = o[t][2 * h];
-        merge_o[(warp * 16 + r) * EV + t * 8 + cq + 1] = o[t][2 * h + 1];
+        merge_o[(wq * 16 + r) * EV + t * 8 + cq] = o[t][2 * h];
+        merge_o[(wq * 16 + r) * EV + t * 8 + cq + 1] = o[t][2 * h + 1];
       }
     }
-    consumer_bar();
+  };
+  auto flush = [&](long long u) {
+    if constexpr (NGRP == 2) {
+      // group 1 hands its state to group 0 through the buffer: warp wq of group 0 merges slot
+      // wq (the same keys of the other chunks) into its registers
+      if (grp == 1) store_state();
+      consumer_bar<NCT>();
+      if (grp == 0) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int r = rA + 8 * h;
+          float l = l_run[h];
+          l += __shfl_xor_sync(0xffffffffu, l, 1);
+          l += __shfl_xor_sync(0xffffffffu, l, 2);
+          const float m1 = merge_ml[(wq * 16 + r) * 2 + 0], l1 = merge_ml[(wq * 16 + r) * 2 + 1];
+          const float M = fmaxf(m_run[h], m1);
+          const float a0 = m_run[h] == -INFINITY ? 0.f : ex2(m_run[h] - M);
+          const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
+#pragma unroll
+          for (int t = 0; t < EV / 8; ++t) {
+            o[t][2 * h] = fmaf(o[t][2 * h], a0, a1 * merge_o[(wq * 16 + r) * EV + t * 8 + cq]);
+            o[t][2 * h + 1] = fmaf(o[t][2 * h + 1], a0, a1 * merge_o[(wq * 16 + r) * EV + t * 8 + cq + 1]);
+          }
+          m_run[h] = M;
+          // the merged row sum, held by lane 0 of the quad so that the next quad sum restores it
+          l_run[h] = (lane & 3) == 0 ? fmaf(l, a0, l1 * a1) : 0.f;
+        }
+      }
+      consumer_bar<NCT>();
+    }
+    if (grp == 0) store_state();
+    consumer_bar<NCT>();
     const size_t slot = static_cast<size_t>(blockIdx.x) + static_cast<size_t>(u);
-    for (int x = threadIdx.x; x < p.R * EV; x += DWARPS * 32) {
+    for (int x = threadIdx.x; x < p.R * EV; x += NCT) {
       const int r = x / EV, e = x % EV;
       float M = -INFINITY;
 #pragma unroll
@@ -452,33 +514,34 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
     // the CTA that finishes the unit's last segment merges all of its partials:
     // publish this partial, count it, and let the count's last arrival combine
     __threadfence();
-    consumer_bar();
+    consumer_bar<NCT>();
     if (threadIdx.x == 0) {
       unsigned int* counters = reinterpret_cast<unsigned int*>(p.ws_ml + (static_cast<size_t>(p.G) + p.n_units) * 32);
       const long long nseg = cta_of(u * p.nc + p.nc - 1, p.T, p.G) - cta_of(u * p.nc, p.T, p.G) + 1;
       *last_flag = atomicAdd(counters + u, 1u) == static_cast<unsigned int>(nseg - 1) ? 1 : 0;
     }
-    consumer_bar();
+    consumer_bar<NCT>();
     if (*last_flag) {
       __threadfence();
-      for (int r = warp; r < p.R; r += DWARPS) combine_row<EV>(p, u, r, lane);
+      for (int r = warp; r < p.R; r += NCW) combine_row<EV>(p, u, r, lane);
     }
-    consumer_bar();
+    consumer_bar<NCT>();
   };
 
-  for (long long c = c_begin; c < c_end; ++c) {
-    const long long u = c / p.nc;
-    if (u != cur_unit) {
-      if (cur_unit >= 0) flush(cur_unit);
-      cur_unit = u;
-      load_q(u);
-      reset_state();
-      if constexpr (EXT) {
-        const int n = static_cast<int>(u / p.H);
-        ks_u = ga.kv_start ? __ldg(ga.kv_start + n) : 0;
-        ke_u = ga.kv_end ? __ldg(ga.kv_end + n) : p.S;
-      }
+  // the units of this CTA's chunk range in order; every consumer warp walks all of them and
+  // meets the others at each unit's flush
+  for (long long cu = c_begin; cu < c_end;) {
+    const long long u = cu / p.nc;
+    const long long cu_end = min(c_end, (u + 1) * p.nc);
+    load_q(u);
+    reset_state();
+    if constexpr (EXT) {
+      const int n = static_cast<int>(u / p.H);
+      ks_u = ga.kv_start ? __ldg(ga.kv_start + n) : 0;
+      ke_u = ga.kv_end ? __ldg(ga.kv_end + n) : p.S;
     }
+    const int first = (grp - static_cast<int>((cu - c_begin) % NGRP) + NGRP) % NGRP;
+  for (long long c = cu + first; c < cu_end; c += NGRP) {
     const int idx = static_cast<int>(c - c_begin);
     const int s = idx % C::NSTAGE;
     const bool w_ok = mbar_wait(full_bar(s), (idx / C::NSTAGE) & 1);
@@ -489,7 +552,7 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
     }
     const uint32_t kbuf = sb + C::OFF_STAGES + s * C::STAGE_BYTES;
     const uint32_t vbuf = kbuf + C::K_BYTES;
-    const int j0 = warp * 16;  // this warp's keys within the chunk
+    const int j0 = wq * 16;  // this warp's keys within the chunk
     const int key0 = GATHER ? 0 : chunk_key0<STREAM>(p, static_cast<int>(c % p.nc)) + j0;
     const int* keys_c = reinterpret_cast<const int*>(sp + C::OFF_KEYS) + s * DC + j0;  // GATHER
 
@@ -602,9 +665,11 @@ __global__ void __launch_bounds__(GATHER ? (DWARPS + GWARPS) * 32 : DTHREADS, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));
   }
-  ok = __all_sync(0xffffffffu, ok);
-  // all four consumer warps always reach this point together (same chunk list)
-  if (ok && cur_unit >= 0) flush(cur_unit);
+    // all consumer warps decide together: a failed wait in any of them ends the walk
+    if (!consumer_bar_and<NCT>(ok)) break;
+    flush(u);
+    cu = cu_end;
+  }
 }
 
 struct DecodePlan {

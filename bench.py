@@ -57,8 +57,8 @@ FFMA_PER_CLK_SM = 122
 NCU_TRAFFIC_BYTES = {
     "dot_causal_2k_bf16": (132_508_416 + 11_135_232, 4),          # prefill_kernel<128,128,dot> (plain variant)
     "dot_causal_2k_bf16:backward": (453_969_920 + 291_908_608, 4),  # bwd_kernel<128,128> (--backward)
-    # decode_partial_kernel<128,128> with the fused combine (a batch-2 capture: 16 GB of cache at batch 32)
-    "decode_sink_gqa_128k_bf16": (1_073_880_576 + 3_166_976, 2),
+    # decode_partial_kernel<128,128>, two consumer groups (a batch-2 capture: 16 GB of cache at batch 32)
+    "decode_sink_gqa_128k_bf16": (1_073_873_920 + 3_484_160, 2),
 }
 
 

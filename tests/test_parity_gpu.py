@@ -104,6 +104,11 @@ DECODE_CASES = [
     R("d_stream_L2_S50_keep0_w10", L=2, S=50, mask_kind="streaming", window=10, keep=0),
     R("d_stream_many_units", L=1, S=3000, N=40, Hq=16, H=8, E=128, Ev=128, mask_kind="streaming", window=256,
       keep=4, scale=0.0884),
+    # units of one 64-key chunk: a CTA's range holds whole units with a single chunk, so one of the two
+    # consumer groups has no chunk of the unit and merges its empty state; two-chunk units with a
+    # ragged second chunk split between CTAs at odd offsets
+    R("d_single_chunk_units_E128", L=1, S=64, N=40, Hq=32, H=8, E=128, Ev=128, sink="normal", scale=0.0884),
+    R("d_two_chunk_ragged_units_E128", L=1, S=100, N=37, Hq=16, H=4, E=128, Ev=128, mode="rbf", scale=0.05),
     # the RBF score on the split-key path (key norms from the staged chunk)
     R("d_rbf_L1_g4_S1000_sink", L=1, S=1000, E=128, Ev=128, N=2, Hq=8, H=2, mode="rbf", sink="normal",
       scale=0.0884),

@@ -18,7 +18,7 @@
 // One CTA per (batch, KV head, 128-key tile) walks the 64-query tiles of every
 // query head of its KV group that can see the key tile, so dK and dV accumulate
 // in tensor memory and are stored once; dQ is accumulated in global memory with
-// reductions.  Per query tile b = it % 2 (two tiles in flight) five tcgen05 MMAs,
+// bulk tensor reduce-adds.  Per query tile b = it % 2 (two tiles in flight) five tcgen05 MMAs,
 // M = 128 keys (or head dimensions for dQ^T):
 //   S^T  = K Q^T      (SS, N = 64)             into TMEM columns S_b = [64 b, 64 b + 64)
 //   dP^T = V dO^T     (SS, N = 64)             into DP_b = [128 + 64 b, 192 + 64 b)
@@ -28,16 +28,18 @@
 // with dS' = dS / c_q; the factor c_q is applied where dQ and dK leave the kernel.
 // dS'^T (128 keys x 64 queries, bf16) is written to shared memory once per tile
 // (two buffers): read K-major it is the A operand of dK, read MN-major the B
-// operand of dQ^T.  dQ^T puts a head-dimension index on each TMEM lane, so one
-// reduction instruction of a warp covers 32 consecutive floats of a dQ row.  dV
+// operand of dQ^T.  dQ^T puts a head-dimension index on each TMEM lane; the readout
+// warpgroup stages it in shared memory as fp32 [query][E] and adds each 32-query half
+// into dq with one bulk tensor reduce-add (the tensor map drops rows past L).  dV
 // and dK live in [256, 256 + Ev) and [256 + Ev, 256 + Ev + E).  tcgen05 MMAs of
 // one thread run in issue order, so S^T of tile it + 2 may be issued into the
 // columns the dV MMA of tile it still reads.
 //
 // Warps: 0-7 compute in two warpgroups (thread = TMEM lane = key row; warpgroup g
 // takes queries [32 g, 32 g + 32) of each tile), 8-11 read dQ^T out (thread =
-// head-dimension index), 12 TMA producer (Q, dO and the tile's lse2 and D), 13
-// MMA issuer.  Every wait is bounded.
+// head-dimension index; their elected thread also issues the dP^T that reuses the
+// columns just read), 12 TMA producer (Q, dO and the tile's lse2 and D), 13 the MMA
+// issuer of dQ^T, 14 the MMA issuer of S^T, dV and dK.  Every wait is bounded.
 
 #include <climits>
 #include <cstdint>

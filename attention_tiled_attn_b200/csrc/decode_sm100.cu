@@ -20,11 +20,12 @@
 // ||k||^2 of its 16 keys from the staged K chunk.
 //
 // Per CTA: one TMA producer warp streams K and V chunks (3-D tensor maps,
-// 128-byte swizzle, zero fill past S) through a ring of stages; four consumer
-// warps each take 16 keys of every chunk.  The query rows of a unit (the
+// 128-byte swizzle, zero fill past S) through a ring of stages; two groups of
+// four consumer warps take alternate chunks (one group in the listed-key variant),
+// each warp 16 keys of its group's chunks.  The query rows of a unit (the
 // Hq/H heads of the KV group times L positions, at most 16) form the M = 16
 // side of mma.sync m16n8k16 products: S = Q K^T, then O += P V with P kept
-// in registers.  Each warp keeps its own online-softmax state; the four are
+// in registers.  Each warp keeps its own online-softmax state; the states are
 // merged through shared memory at the end of a segment.
 //
 // Masks follow the bottom-right alignment of page "SDPA란 무엇인가" §4
